@@ -1,0 +1,143 @@
+"""CPU oracle for the RT-Lynx activation-sparse linear layer (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA product path never does.
+
+The arithmetic lives in ``rtlynx_oracle.c`` (plain C, double precision, plain
+triple-loop GEMMs, OpenMP over tokens).  It follows the four-step pipeline
+paragraph of the RT-Lynx summary page (paper.rainbus.top, arXiv 2605.26632),
+steps 1-3: Top-K 2-of-4 mask, norm-compensating scale s, LoRA branch on the
+dense X, and the dense path for skipped layers.  This module only compiles the
+C file with gcc and marshals numpy arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rtlynx_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lib = None
+
+MODE_SPARSE = 0
+MODE_DENSE_SKIP = 1
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle C source into a shared library (gcc, OpenMP)."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, src, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns as numpy uint16")
+    return a
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """ctypes view of one compiled oracle library."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        p = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.oracle_sparsify.argtypes = [p, i64, i64, p, p, p]
+        lib.oracle_sparsify.restype = ctypes.c_int
+        lib.oracle_linear_rows.argtypes = [p, p, p, p, i64, i64, i64, i64, ctypes.c_int, p, i64, p, p]
+        lib.oracle_linear_rows.restype = ctypes.c_int
+        lib.oracle_bf16_from_double.argtypes = [ctypes.c_double]
+        lib.oracle_bf16_from_double.restype = ctypes.c_uint16
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        self.lib = lib
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    def bf16_round(self, v: float) -> int:
+        """bf16 bits of the double v, rounded to nearest, ties to even."""
+        return int(self.lib.oracle_bf16_from_double(float(v)))
+
+    def sparsify(self, X: np.ndarray):
+        """Step 1 per token: (meta [M,K/4] uint8, vals [M,K/2] bf16 bits, s [M] float32)."""
+        X = _u16(X)
+        M, K = X.shape
+        meta = np.empty((M, K // 4), np.uint8)
+        vals = np.empty((M, K // 2), np.uint16)
+        s = np.empty((M,), np.float32)
+        rc = self.lib.oracle_sparsify(_ptr(X), M, K, _ptr(meta), _ptr(vals), _ptr(s))
+        if rc:
+            raise ValueError("oracle_sparsify rejected its arguments")
+        return meta, vals, s
+
+    def linear(self, X, W, L_A=None, L_B=None, mode: int = MODE_SPARSE, rows=None, want_T: bool = False):
+        """Y (float64) for the listed rows (all rows when rows is None); also T when want_T."""
+        X = _u16(X)
+        W = _u16(W)
+        M, K = X.shape
+        N = W.shape[0]
+        if W.shape[1] != K:
+            raise ValueError("W must be [D_out, D_in]")
+        R = 0
+        if L_A is not None and L_B is not None:
+            L_A = _u16(L_A)
+            L_B = _u16(L_B)
+            R = L_B.shape[0]
+            if L_A.shape != (N, R) or L_B.shape != (R, K):
+                raise ValueError("L_A must be [D_out,R] and L_B [R,D_in]")
+        else:
+            L_A = L_B = None
+        if rows is None:
+            rows_arr = None
+            nrows = M
+        else:
+            rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+            nrows = rows_arr.shape[0]
+        Y = np.empty((nrows, N), np.float64)
+        T = np.empty((nrows, max(R, 1)), np.float64) if want_T else None
+        rc = self.lib.oracle_linear_rows(_ptr(X), _ptr(W), _ptr(L_A), _ptr(L_B), M, K, N, R, int(mode),
+                                         _ptr(rows_arr), nrows, _ptr(Y), _ptr(T))
+        if rc:
+            raise ValueError("oracle_linear_rows rejected its arguments")
+        if want_T:
+            return Y, T[:, :R]
+        return Y
+
+
+def _default() -> Oracle:
+    global _lib
+    if _lib is None:
+        _lib = Oracle(build())
+    return _lib
+
+
+def num_threads() -> int:
+    return _default().num_threads()
+
+
+def bf16_round(v: float) -> int:
+    return _default().bf16_round(v)
+
+
+def sparsify(X):
+    return _default().sparsify(X)
+
+
+def linear(X, W, L_A=None, L_B=None, mode: int = MODE_SPARSE, rows=None, want_T: bool = False):
+    return _default().linear(X, W, L_A, L_B, mode=mode, rows=rows, want_T=want_T)

@@ -1,0 +1,217 @@
+/*
+ * CPU oracle for the RT-Lynx activation-sparse linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, __graft_entry__.smoke() and the
+ * CPU-baseline leg of bench.py may load this library.  The product path (the
+ * CUDA library under activation_sparse_gemm_b200/) shares no code with it and
+ * never calls it.
+ *
+ * What it computes (RT-Lynx, paper.rainbus.top summary of arXiv 2605.26632,
+ * "four-step pipeline" paragraph, steps 1-2; the fugumt abstract page for the
+ * same paper states the method's scope):
+ *
+ *   X~   = per token, keep 2 of every 4 consecutive channels (Top-K, 2 of 4)
+ *   s    = ||X||_2 / (||X~||_2 + eps),  eps = 1e-8
+ *   S(X) = s * X~
+ *   Y_s  = S(X) W^T,   Y_r = X (L_A L_B)^T  (dense X, rank R),   Y = Y_s + Y_r
+ *   dense-skip layers ("Selective Layer Skipping", step 3): Y = X W^T
+ *
+ * Readings where the page is silent (each is listed in the design notes):
+ *   - Top-K ranks by magnitude |x|; equal magnitudes go to the lower index;
+ *     -0 and +0 are equal.  An all-zero group keeps indices 0 and 1.
+ *   - eps is added to the norm (not to its square), as printed.
+ *   - s is a float32 per token: computed here in double, rounded once.
+ *   - the stored sparse value is bf16_rne(s * x), from the exact product.
+ *   - the LoRA branch sees the dense X; no alpha/r scale, no bias.
+ *   - metadata nibble for a group = i0 | (i1 << 2) with i0 < i1 (the
+ *     2:4 encoding of the sparse tensor-core instructions).
+ *
+ * All arithmetic on values is double; every GEMM is a plain triple loop with
+ * no blocking or reordering; rows are independent and run under OpenMP.
+ *
+ * Layouts (row-major, little-endian, bf16 passed as uint16 bit patterns):
+ *   X [M,K], W [N,K], L_A [N,R], L_B [R,K]
+ *   meta [M, K/4] uint8 (one nibble per byte), vals [M, K/2] bf16, s [M] f32
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define RTLYNX_EPS 1e-8
+
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16, ties to even, in one step (no detour
+ * through float, so there is no double rounding).  bf16 has 8 significant
+ * bits and float's exponent range; its subnormals are multiples of 2^-133. */
+static uint16_t double_to_bf16_rne(double v)
+{
+    double a = fabs(v);
+    double r;
+    if (a == 0.0) {
+        r = 0.0;
+    } else if (a < 0x1p-126) {
+        r = ldexp(nearbyint(ldexp(a, 133)), -133);
+    } else {
+        int e;
+        double m = frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+        r = ldexp(nearbyint(ldexp(m, 8)), e - 8);
+    }
+    float f = (float)r; /* exact, or +inf past the largest bf16 */
+    if (v < 0 || (v == 0 && signbit(v))) f = -f;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+uint16_t oracle_bf16_from_double(double v) { return double_to_bf16_rne(v); }
+double oracle_double_from_bf16(uint16_t b) { return bf16_to_double(b); }
+
+/* Top-K (2 of 4) on one group: index i is kept iff fewer than two other
+ * entries beat it, where j beats i when |x_j| > |x_i|, or |x_j| == |x_i|
+ * and j < i.  Returns the kept indices in ascending order. */
+static void keep_two_of_four(const double x[4], int *i0, int *i1)
+{
+    int kept[2], n = 0;
+    for (int i = 0; i < 4; ++i) {
+        int beaten = 0;
+        for (int j = 0; j < 4; ++j) {
+            if (j == i) continue;
+            double aj = fabs(x[j]), ai = fabs(x[i]);
+            if (aj > ai || (aj == ai && j < i)) ++beaten;
+        }
+        if (beaten < 2) kept[n++] = i;
+    }
+    *i0 = kept[0];
+    *i1 = kept[1];
+}
+
+/* Step 1 for one token: mask, norms, s, and the rounded kept values.
+ * Xrow [K] bf16 -> meta [K/4], vals [K/2] bf16, returns s; also writes the
+ * dense S(X) row (double, zeros at dropped positions) when S != NULL. */
+static float sparsify_row(const uint16_t *Xrow, int64_t K, uint8_t *meta,
+                          uint16_t *vals, double *S)
+{
+    double nx = 0.0, nt = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double x = bf16_to_double(Xrow[k]);
+        nx += x * x;
+    }
+    for (int64_t g = 0; g < K / 4; ++g) {
+        double x[4];
+        for (int i = 0; i < 4; ++i) x[i] = bf16_to_double(Xrow[4 * g + i]);
+        int i0, i1;
+        keep_two_of_four(x, &i0, &i1);
+        nt += x[i0] * x[i0] + x[i1] * x[i1];
+    }
+    float s = (float)(sqrt(nx) / (sqrt(nt) + RTLYNX_EPS));
+    for (int64_t g = 0; g < K / 4; ++g) {
+        double x[4];
+        for (int i = 0; i < 4; ++i) x[i] = bf16_to_double(Xrow[4 * g + i]);
+        int i0, i1;
+        keep_two_of_four(x, &i0, &i1);
+        uint16_t v0 = double_to_bf16_rne((double)s * x[i0]);
+        uint16_t v1 = double_to_bf16_rne((double)s * x[i1]);
+        if (meta) meta[g] = (uint8_t)(i0 | (i1 << 2));
+        if (vals) {
+            vals[2 * g] = v0;
+            vals[2 * g + 1] = v1;
+        }
+        if (S) {
+            for (int i = 0; i < 4; ++i) S[4 * g + i] = 0.0;
+            S[4 * g + i0] = bf16_to_double(v0);
+            S[4 * g + i1] = bf16_to_double(v1);
+        }
+    }
+    return s;
+}
+
+/* Mask, metadata, s and compressed values for every token. */
+int oracle_sparsify(const uint16_t *X, int64_t M, int64_t K, uint8_t *meta,
+                    uint16_t *vals, float *s)
+{
+    if (M < 0 || K <= 0 || K % 4) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t m = 0; m < M; ++m) {
+        float sm = sparsify_row(X + m * K, K, meta ? meta + m * (K / 4) : NULL,
+                                vals ? vals + m * (K / 2) : NULL, NULL);
+        if (s) s[m] = sm;
+    }
+    return 0;
+}
+
+/* Y rows (and optionally T rows) for the tokens listed in rows[0..nrows)
+ * (rows == NULL means every token, nrows = M).
+ *   mode 0 (sparse):     T = X L_B^T,  Y = S(X) W^T + T L_A^T
+ *   mode 1 (dense-skip): Y = X W^T
+ * Y [nrows, N] double, T [nrows, R] double (may be NULL). R == 0 or a NULL
+ * L_A / L_B means no LoRA branch. */
+int oracle_linear_rows(const uint16_t *X, const uint16_t *W, const uint16_t *L_A,
+                       const uint16_t *L_B, int64_t M, int64_t K, int64_t N,
+                       int64_t R, int mode, const int64_t *rows, int64_t nrows,
+                       double *Y, double *T)
+{
+    if (M < 0 || K <= 0 || N <= 0 || R < 0 || (mode != 0 && mode != 1)) return 1;
+    if (mode == 0 && K % 4) return 1;
+    if (!rows) nrows = M;
+    int use_lora = (mode == 0 && R > 0 && L_A && L_B);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) {
+            bad = 1;
+            continue;
+        }
+        const uint16_t *Xrow = X + m * K;
+        double *A = (double *)malloc(sizeof(double) * (size_t)K);
+        double *Trow = (double *)malloc(sizeof(double) * (size_t)(R > 0 ? R : 1));
+        if (mode == 0) {
+            sparsify_row(Xrow, K, NULL, NULL, A);
+        } else {
+            for (int64_t k = 0; k < K; ++k) A[k] = bf16_to_double(Xrow[k]);
+        }
+        if (use_lora) {
+            for (int64_t r = 0; r < R; ++r) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += bf16_to_double(Xrow[k]) * bf16_to_double(L_B[r * K + k]);
+                Trow[r] = acc;
+            }
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += A[k] * bf16_to_double(W[n * K + k]);
+            if (use_lora) {
+                double lr = 0.0;
+                for (int64_t r = 0; r < R; ++r) lr += Trow[r] * bf16_to_double(L_A[n * R + r]);
+                acc += lr;
+            }
+            Y[i * N + n] = acc;
+        }
+        if (T && R > 0) {
+            for (int64_t r = 0; r < R; ++r) T[i * R + r] = use_lora ? Trow[r] : 0.0;
+        }
+        free(A);
+        free(Trow);
+    }
+    return bad ? 1 : 0;
+}
+
+/* Threads the OpenMP runtime will use (reported next to CPU timings). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
