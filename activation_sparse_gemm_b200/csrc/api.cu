@@ -1,0 +1,378 @@
+// C ABI of the RT-Lynx linear layer: argument checks, workspace management,
+// tensor-map encoding and the launch sequence.  See include/rtlynx.h.
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/rtlynx.h"
+#include "internal.h"
+
+namespace rtlynx {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    bool supported = false;
+    int num_sms = 0;
+    int* err_word = nullptr;  // device memory, one int
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+struct WsEntry {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+struct WsKey {
+    int dev;
+    cudaStream_t stream;
+    bool operator==(const WsKey& o) const { return dev == o.dev && stream == o.stream; }
+};
+struct WsKeyHash {
+    size_t operator()(const WsKey& k) const {
+        return std::hash<void*>()(static_cast<void*>(k.stream)) ^ (static_cast<size_t>(k.dev) << 1);
+    }
+};
+std::unordered_map<WsKey, WsEntry, WsKeyHash> g_ws;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int current_device(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RTLYNX_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.init) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return RTLYNX_ERR_CUDA;
+        di.supported = (major == 10 && minor == 0);
+        di.num_sms = sms;
+        if (di.supported) {
+            if (cudaMalloc(&di.err_word, sizeof(int)) != cudaSuccess) return RTLYNX_ERR_OOM;
+            if (cudaMemset(di.err_word, 0, sizeof(int)) != cudaSuccess) return RTLYNX_ERR_CUDA;
+        }
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return RTLYNX_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        di.init = true;
+    }
+    if (!di.supported) return RTLYNX_ERR_UNSUPPORTED;
+    *out = &di;
+    return RTLYNX_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int validate(const void* X, const void* W, const void* L_A, const void* L_B, const void* Y, int64_t M,
+             int64_t K, int64_t N, int64_t R, int mode) {
+    if (mode != RTLYNX_MODE_SPARSE && mode != RTLYNX_MODE_DENSE_SKIP) return RTLYNX_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0 || N <= 0 || R < 0) return RTLYNX_ERR_INVALID_ARG;
+    if (K % 8 != 0 || N % 8 != 0) return RTLYNX_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31) - kBM || K > (int64_t(1) << 30) || N > (int64_t(1) << 30))
+        return RTLYNX_ERR_UNSUPPORTED;
+    if (!X || !W || !Y) return RTLYNX_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(Y)) return RTLYNX_ERR_INVALID_ARG;
+    if (mode == RTLYNX_MODE_SPARSE && R > 0) {
+        if (!L_A || !L_B) return RTLYNX_ERR_INVALID_ARG;
+        if (!aligned16(L_A) || !aligned16(L_B)) return RTLYNX_ERR_INVALID_ARG;
+        if (R % 8 != 0 || R > 256) return RTLYNX_ERR_UNSUPPORTED;
+    }
+    return RTLYNX_OK;
+}
+
+}  // namespace
+
+int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swizzle) {
+    if (!g_encode) return cudaErrorInitializationError;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
+}
+
+Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
+    Dims d;
+    d.M = M;
+    d.K = K;
+    d.N = N;
+    d.R = R;
+    d.M_pad = (M + kBM - 1) / kBM * kBM;
+    d.m_blocks = d.M_pad / kBM;
+    d.k_tiles = (K + kBK - 1) / kBK;
+    d.k_chunks = (K + kChunkK - 1) / kChunkK;
+    d.Kc_pad = d.k_tiles * (kBK / 2);
+    d.R_pad = R > 0 ? (R + 31) / 32 * 32 : 0;
+    // Enough CTAs in the norm / LoRA-down pass to cover the GPU about twice,
+    // every split holding at least one K tile.
+    int64_t target = 2 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148);
+    int64_t ns = (target + d.m_blocks - 1) / d.m_blocks;
+    if (ns < 1) ns = 1;
+    if (ns > d.k_tiles) ns = d.k_tiles;
+    const int64_t tps = (d.k_tiles + ns - 1) / ns;
+    d.nsplit = (d.k_tiles + tps - 1) / tps;
+    return d;
+}
+
+WsLayout make_ws_layout(const Dims& d) {
+    WsLayout l;
+    size_t off = 0;
+    l.vals = off;
+    off = align256(off + static_cast<size_t>(d.M_pad) * d.Kc_pad * 2);
+    l.meta = off;
+    off = align256(off + static_cast<size_t>(d.m_blocks) * d.k_chunks * kChunkBytes);
+    l.s = off;
+    off = align256(off + static_cast<size_t>(d.M_pad) * 4);
+    l.T = off;
+    off = align256(off + static_cast<size_t>(d.M_pad) * d.R_pad * 2);
+    l.part_norm = off;
+    off = align256(off + static_cast<size_t>(d.nsplit) * d.M_pad * 2 * 8);
+    l.part_T = off;
+    off = align256(off + static_cast<size_t>(d.nsplit) * d.M_pad * d.R_pad * 4);
+    l.total = off;
+    return l;
+}
+
+static Workspace carve(void* base, const WsLayout& l) {
+    uint8_t* b = static_cast<uint8_t*>(base);
+    Workspace w;
+    w.vals = reinterpret_cast<uint16_t*>(b + l.vals);
+    w.meta = b + l.meta;
+    w.s = reinterpret_cast<float*>(b + l.s);
+    w.T = reinterpret_cast<uint16_t*>(b + l.T);
+    w.part_norm = reinterpret_cast<double*>(b + l.part_norm);
+    w.part_T = reinterpret_cast<float*>(b + l.part_T);
+    return w;
+}
+
+// Grow (or create) the cached workspace of (device, stream).
+static int cached_workspace(int dev, cudaStream_t stream, size_t bytes, void** out) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    WsEntry& e = g_ws[WsKey{dev, stream}];
+    if (e.bytes < bytes) {
+        if (e.ptr) {
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return RTLYNX_ERR_CUDA;
+            cudaFree(e.ptr);
+            e.ptr = nullptr;
+            e.bytes = 0;
+        }
+        if (cudaMalloc(&e.ptr, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return RTLYNX_ERR_OOM;
+        }
+        e.bytes = bytes;
+    }
+    *out = e.ptr;
+    return RTLYNX_OK;
+}
+
+static int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
+                        cudaStream_t stream) {
+    if (launch_norms_lora_down(d, X, L_B, ws, err, stream)) return RTLYNX_ERR_CUDA;
+    if (launch_compress(d, X, ws, stream)) return RTLYNX_ERR_CUDA;
+    return RTLYNX_OK;
+}
+
+}  // namespace rtlynx
+
+using namespace rtlynx;
+
+extern "C" {
+
+size_t rtlynx_workspace_size(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode) {
+    if (mode == RTLYNX_MODE_DENSE_SKIP) return 0;
+    if (mode != RTLYNX_MODE_SPARSE || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8)
+        return 0;
+    DeviceInfo* di = nullptr;
+    const int sms = current_device(&di) == RTLYNX_OK ? di->num_sms : 148;
+    return make_ws_layout(make_dims(M, D_in, D_out, R, sms)).total;
+}
+
+int rtlynx_workspace_layout(int64_t M, int64_t D_in, int64_t D_out, int64_t R, rtlynx_ws_layout* out) {
+    if (!out || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8) return RTLYNX_ERR_INVALID_ARG;
+    DeviceInfo* di = nullptr;
+    const int sms = current_device(&di) == RTLYNX_OK ? di->num_sms : 148;
+    const Dims d = make_dims(M, D_in, D_out, R, sms);
+    const WsLayout l = make_ws_layout(d);
+    out->M_pad = d.M_pad;
+    out->Kc_pad = d.Kc_pad;
+    out->k_chunks = d.k_chunks;
+    out->R_pad = d.R_pad;
+    out->vals = l.vals;
+    out->meta = l.meta;
+    out->s = l.s;
+    out->T = l.T;
+    out->total = l.total;
+    return RTLYNX_OK;
+}
+
+int rtlynx_linear_ws_events(const void* X, const void* W, const void* L_A, const void* L_B, void* Y,
+                            int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* workspace,
+                            size_t ws_bytes, void* ev_start, void* ev_mid, void* ev_end, void* stream_) {
+    int rc = validate(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode);
+    if (rc) return rc;
+    DeviceInfo* di = nullptr;
+    rc = current_device(&di);
+    if (rc) return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool lora = (mode == RTLYNX_MODE_SPARSE) && R > 0 && L_A && L_B;
+    const Dims d = make_dims(M, D_in, D_out, lora ? R : 0, di->num_sms);
+    auto record = [&](void* ev) {
+        return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev), stream) == cudaSuccess;
+    };
+    if (mode == RTLYNX_MODE_DENSE_SKIP) {
+        Workspace none{};
+        if (!record(ev_start) || !record(ev_mid)) return RTLYNX_ERR_CUDA;
+        if (launch_gemm(d, false, X, W, nullptr, none, Y, di->num_sms, di->err_word, stream)) return RTLYNX_ERR_CUDA;
+        return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+    }
+    const WsLayout l = make_ws_layout(d);
+    if (!workspace || ws_bytes < l.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return RTLYNX_ERR_INVALID_ARG;
+    const Workspace ws = carve(workspace, l);
+    if (!record(ev_start)) return RTLYNX_ERR_CUDA;
+    rc = run_prologue(d, X, lora ? L_B : nullptr, ws, di->err_word, stream);
+    if (rc) return rc;
+    if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
+    if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, di->num_sms, di->err_word, stream))
+        return RTLYNX_ERR_CUDA;
+    return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+}
+
+int rtlynx_linear_ws(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
+                     int64_t D_in, int64_t D_out, int64_t R, int mode, void* workspace, size_t ws_bytes,
+                     void* stream_) {
+    return rtlynx_linear_ws_events(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, workspace, ws_bytes, nullptr,
+                                   nullptr, nullptr, stream_);
+}
+
+int rtlynx_linear(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
+                  int64_t D_in, int64_t D_out, int64_t R, int mode, void* stream_) {
+    int rc = validate(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode);
+    if (rc) return rc;
+    DeviceInfo* di = nullptr;
+    rc = current_device(&di);
+    if (rc) return rc;
+    if (mode == RTLYNX_MODE_DENSE_SKIP)
+        return rtlynx_linear_ws(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, nullptr, 0, stream_);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool lora = R > 0 && L_A && L_B;
+    const size_t bytes = make_ws_layout(make_dims(M, D_in, D_out, lora ? R : 0, di->num_sms)).total;
+    void* ws = nullptr;
+    rc = cached_workspace(dev, static_cast<cudaStream_t>(stream_), bytes, &ws);
+    if (rc) return rc;
+    return rtlynx_linear_ws(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, ws, bytes, stream_);
+}
+
+int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_in, int64_t R, void* vals,
+                          void* meta, void* s, void* T, void* stream_) {
+    if (!X || M <= 0 || D_in <= 0 || D_in % 8 || R < 0 || !aligned16(X)) return RTLYNX_ERR_INVALID_ARG;
+    if (R > 0 && (!L_B || !aligned16(L_B))) return RTLYNX_ERR_INVALID_ARG;
+    if (R % 8 != 0 || R > 256) return RTLYNX_ERR_UNSUPPORTED;
+    DeviceInfo* di = nullptr;
+    int rc = current_device(&di);
+    if (rc) return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const Dims d = make_dims(M, D_in, 8, R, di->num_sms);
+    const WsLayout l = make_ws_layout(d);
+    void* base = nullptr;
+    rc = cached_workspace(dev, stream, l.total, &base);
+    if (rc) return rc;
+    const Workspace ws = carve(base, l);
+    rc = run_prologue(d, X, R > 0 ? L_B : nullptr, ws, di->err_word, stream);
+    if (rc) return rc;
+    if (launch_unpack_debug(d, ws, vals, meta, s, R > 0 ? T : nullptr, stream)) return RTLYNX_ERR_CUDA;
+    return RTLYNX_OK;
+}
+
+int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const void* L_B, void* Y_host,
+                       int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* X_dev, void* Y_dev,
+                       void* stream_) {
+    if (!X_host || !Y_host) return RTLYNX_ERR_INVALID_ARG;
+    int rc = validate(X_dev, W, L_A, L_B, Y_dev, M, D_in, D_out, R, mode);
+    if (rc) return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(M) * D_in * 2, cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess)
+        return RTLYNX_ERR_CUDA;
+    rc = rtlynx_linear(X_dev, W, L_A, L_B, Y_dev, M, D_in, D_out, R, mode, stream_);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(M) * D_out * 2, cudaMemcpyDeviceToHost, stream) !=
+        cudaSuccess)
+        return RTLYNX_ERR_CUDA;
+    return RTLYNX_OK;
+}
+
+int rtlynx_stream_status(void* stream_) {
+    DeviceInfo* di = nullptr;
+    int rc = current_device(&di);
+    if (rc) return rc;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream_)) != cudaSuccess) return RTLYNX_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, di->err_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RTLYNX_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemset(di->err_word, 0, sizeof(int)) != cudaSuccess) return RTLYNX_ERR_CUDA;
+        return RTLYNX_ERR_DEVICE_TIMEOUT;
+    }
+    return RTLYNX_OK;
+}
+
+const char* rtlynx_status_string(int status) {
+    switch (status) {
+        case RTLYNX_OK: return "ok";
+        case RTLYNX_ERR_INVALID_ARG: return "invalid argument";
+        case RTLYNX_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case RTLYNX_ERR_CUDA: return "CUDA call failed";
+        case RTLYNX_ERR_OOM: return "out of device memory";
+        case RTLYNX_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+void rtlynx_release(void) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto& kv : g_ws) {
+        if (kv.second.ptr) {
+            cudaSetDevice(kv.first.dev);
+            cudaDeviceSynchronize();
+            cudaFree(kv.second.ptr);
+        }
+    }
+    g_ws.clear();
+    for (int i = 0; i < kMaxDevices; ++i) {
+        if (g_dev[i].err_word) {
+            cudaSetDevice(i);
+            cudaFree(g_dev[i].err_word);
+        }
+        g_dev[i] = DeviceInfo{};
+    }
+    cudaSetDevice(cur);
+}
+
+}  // extern "C"

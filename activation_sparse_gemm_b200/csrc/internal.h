@@ -1,0 +1,61 @@
+// Declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rtlynx {
+
+// Tile geometry shared by the prologue and the GEMM.
+constexpr int kBM = 128;          // rows (tokens) per tile
+constexpr int kBN = 256;          // output columns per tile
+constexpr int kBK = 64;           // logical K per pipeline stage
+constexpr int kChunkK = 128;      // logical K per metadata chunk (4 sparse MMAs of K = 32)
+constexpr int kChunkBytes = 2048; // 128 lanes x 16 bytes of metadata per chunk
+
+// Sizes derived from one problem.
+struct Dims {
+    int64_t M, K, N, R;
+    int64_t M_pad;        // M rounded up to kBM
+    int64_t m_blocks;     // M_pad / kBM
+    int64_t k_tiles;      // ceil(K / kBK)
+    int64_t k_chunks;     // ceil(K / kChunkK)
+    int64_t Kc_pad;       // compressed row length in elements = k_tiles * kBK / 2
+    int64_t R_pad;        // R rounded up to 32 (0 when R == 0)
+    int64_t nsplit;       // K-splits of the norm / LoRA-down pass
+};
+
+// Byte offsets of the sparse-mode workspace regions (each 256-byte aligned).
+struct WsLayout {
+    size_t vals, meta, s, T, part_norm, part_T, total;
+};
+
+Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms);
+WsLayout make_ws_layout(const Dims& d);
+
+struct Workspace {
+    uint16_t* vals;       // [M_pad, Kc_pad] bf16, compressed kept values (rows >= M are zero)
+    uint8_t* meta;        // [m_blocks, k_chunks, 2048] metadata chunks in tensor-memory order
+    float* s;             // [M_pad] per-token scale
+    uint16_t* T;          // [M_pad, R_pad] bf16, X L_B^T
+    double* part_norm;    // [nsplit, M_pad, 2] partial sum of x^2 and of kept x^2
+    float* part_T;        // [nsplit, M_pad, R_pad] partial X L_B^T
+};
+
+// Tensor-map encoding through the driver entry point (no libcuda link needed).
+int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swizzle);
+
+// Launchers; each returns a cudaError_t value (0 on success).
+int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
+                           cudaStream_t stream);
+int launch_compress(const Dims& d, const void* X, const Workspace& ws, cudaStream_t stream);
+int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
+                void* Y, int num_sms, int* err, cudaStream_t stream);
+int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,
+                        cudaStream_t stream);
+
+}  // namespace rtlynx

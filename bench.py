@@ -1,0 +1,379 @@
+"""Benchmark of the RT-Lynx fused activation-sparse + LoRA linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qkv] [--impl ours|reference]
+
+One step = one call of the whole layer (sparsify prologue with the LoRA
+down-projection, then the sparse GEMM with the LoRA up-projection accumulated
+in the same tensor-memory accumulator) on one batch of tokens resident in HBM.
+L2 is flushed (a 256 MB write) before every timed step; each step is timed
+with CUDA events on the launching stream and the mean over K steps is
+reported; under torchrun the max over ranks is taken.  Every rank processes
+its own token block with the same weights (tokens are independent, so there
+is no data-path collective): scaling is weak.
+
+Prints ONE JSON line (rank 0).  value = dense-equivalent TFLOP/s of the whole
+job: (2*M*D_in*D_out + 2*M*R*(D_in+D_out)) * ranks / time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused 2:4 act-sparse+LoRA linear: µs/call, TFLOP/s, speedup vs dense bf16"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qkv")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def workload_desc(wl):
+    return {"workload": f"{wl.name}: M={wl.M} D_in={wl.D_in} D_out={wl.D_out} R={wl.R}",
+            "M": wl.M, "D_in": wl.D_in, "D_out": wl.D_out, "R": wl.R, "p_out": wl.p_out,
+            "seed": wl.seed, "x_dist": "GELU(N(0,1)*c)" if wl.gelu else "N(0,1)*c, c~LogNormal(0,1), outliers x10"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def oracle_sample(wl, X, W, L_A, L_B, target_s, min_rows=2):
+    """Times the CPU oracle on the first n token rows, n chosen for ~target_s of work."""
+    import oracle
+    n = min_rows
+    t0 = time.perf_counter()
+    oracle.linear(X, W, L_A, L_B, rows=list(range(n)))
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(max(min_rows, min(wl.M, n * target_s / dt)))
+    t0 = time.perf_counter()
+    oracle.linear(X, W, L_A, L_B, rows=list(range(n)))
+    dt = time.perf_counter() - t0
+    flop = 2 * n * wl.D_in * wl.D_out + 2 * n * wl.R * (wl.D_in + wl.D_out)
+    return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {n} of {wl.M} tokens of the {wl.name} workload (all D_out outputs), "
+                      f"{dt:.1f} s wall, fp64 triple loop, OpenMP over tokens"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, torch_device):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            self.samples.append((mhz, reasons))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.005)
+
+    def start(self):
+        self.sample()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        self._t.join()
+        self.sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": getattr(self, "err", "no samples")}
+        mhz = [m for m, _ in self.samples]
+        active = 0
+        for _, r in self.samples:
+            active |= r
+        names = [k for k, v in self.REASONS.items() if active & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(mhz), "sm_mhz_min": min(mhz)}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, wl):
+    from activation_sparse_gemm_b200.inputs import make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    X, W, L_A, L_B = make_inputs(wl)
+    import oracle
+    oracle.build()
+    # rows per step sized so warm-up + K steps stay within a few minutes
+    t0 = time.perf_counter()
+    oracle.linear(X, W, L_A, L_B, rows=[0, 1])
+    per_row = (time.perf_counter() - t0) / 2
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(wl.M, budget / max(per_row, 1e-9))))
+    rows = list(range(n))
+    for _ in range(args.warmup):
+        oracle.linear(X, W, L_A, L_B, rows=rows[:1])
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.linear(X, W, L_A, L_B, rows=rows)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    flop = 2 * n * wl.D_in * wl.D_out + 2 * n * wl.R * (wl.D_in + wl.D_out)
+    value = flop / (ms / 1e3) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_desc(wl),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"first {n} of {wl.M} tokens per step (all D_out outputs)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, wl):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import activation_sparse_gemm_b200 as rl
+    from activation_sparse_gemm_b200.inputs import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    rl.lib()
+
+    X, W, L_A, L_B = make_inputs(wl)
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+    Xd, Wd, Ad, Bd = dev(X), dev(W), dev(L_A), dev(L_B)
+    M, K, N, R = wl.M, wl.D_in, wl.D_out, wl.R
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    ws_bytes = rl.rtlynx_workspace_size(M, K, N, R, rl.MODE_SPARSE)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    def sparse_step(e0=None, e1=None, e2=None, mode=rl.MODE_SPARSE):
+        rl.rtlynx_linear_ws_events(Xd, Wd, Ad, Bd, Y, M, K, N, R, mode, ws, ws_bytes, e0, e1, e2, stream)
+
+    # warm-up (also checks the device error word once)
+    for _ in range(max(args.warmup, 3)):
+        sparse_step()
+    if rl.rtlynx_stream_status(stream) != rl.OK:
+        raise RuntimeError("device-side error during warm-up")
+
+    def timed(fn, steps, n_events=2):
+        """Runs fn(events) steps times with an L2 flush before each; returns per-step event lists."""
+        evs = []
+        for _ in range(steps):
+            flush.fill_(1)
+            es = [ev() for _ in range(n_events)]
+            evs.append(es)
+            fn(es)
+        return evs
+
+    clocks = ClockSampler(device)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    evs = timed(lambda es: sparse_step(es[0], es[1], es[2]), args.steps, 3)
+    torch.cuda.synchronize()
+    clocks.stop()
+    barrier()
+    step_ms = [a.elapsed_time(c) for a, b, c in evs]
+    pro_ms = [a.elapsed_time(b) for a, b, c in evs]
+    gemm_ms = [b.elapsed_time(c) for a, b, c in evs]
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # same-run comparisons (not part of the headline value)
+    for _ in range(3):
+        torch.matmul(Xd, Wd.t(), out=Y)
+    cublas_pairs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a = ev()
+        torch.matmul(Xd, Wd.t(), out=Y)
+        b = ev()
+        cublas_pairs.append((a, b))
+    torch.cuda.synchronize()
+    cublas_ms = statistics.mean(a.elapsed_time(b) for a, b in cublas_pairs)
+    ours_dense_pairs = []
+    for _ in range(max(3, args.warmup)):
+        sparse_step(mode=rl.MODE_DENSE_SKIP)
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a = ev()
+        sparse_step(mode=rl.MODE_DENSE_SKIP)
+        b = ev()
+        ours_dense_pairs.append((a, b))
+    torch.cuda.synchronize()
+    ours_dense_ms = statistics.mean(a.elapsed_time(b) for a, b in ours_dense_pairs)
+
+    # end to end through the host-buffer entry point
+    Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        rl.rtlynx_linear_host(Xh, Wd, Ad, Bd, Yh, M, K, N, R, rl.MODE_SPARSE, Xd, Y, stream)
+    e2e_pairs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a = ev()
+        rl.rtlynx_linear_host(Xh, Wd, Ad, Bd, Yh, M, K, N, R, rl.MODE_SPARSE, Xd, Y, stream)
+        b = ev()
+        e2e_pairs.append((a, b))
+    torch.cuda.synchronize()
+    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_pairs)
+    status = rl.rtlynx_stream_status(stream)
+    if status != rl.OK:
+        raise RuntimeError(f"device-side error: {rl.rtlynx_status_string(status)}")
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flop = wl.dense_equiv_flop
+    value = flop * world / (ms / 1e3) / 1e12
+    gemm_mean = statistics.mean(gemm_ms)
+    gemm_flop = 2 * M * N * K + 2 * M * R * N
+    peaks, peaks_kind = load_peaks()
+    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    achieved = gemm_flop / (gemm_mean / 1e3) / 1e12
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "gemm_sparse_traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            tj = json.load(f)
+        if tj.get("workload") == wl.name and tj.get("kernel_rev") == kernel_rev():
+            traffic = tj.get("dram_bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3,
+        "speedup_vs_dense_bf16": cublas_ms / ms, "dense_bf16_cublas_us": cublas_ms * 1e3,
+        "ours_dense_skip_us": ours_dense_ms * 1e3,
+        "phases_us": {"sparsify_prologue": statistics.mean(pro_ms) * 1e3, "sparse_gemm_lora": gemm_mean * 1e3},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, DiT-shaped; random-init weights)",
+        "config": {**workload_desc(wl), "global_batch": M * world,
+                   "parallelism": f"token blocks, {world} rank(s), no collective",
+                   "l2": "flushed before every timed step (256 MB write)"},
+        "e2e": {"value": flop * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "us_per_call": e2e_ms * 1e3},
+        "gpu_launches": kernels_per_step(R) * args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": sparse_peak, "unit": "TFLOP/s",
+                     "frac": achieved / sparse_peak, "traffic": traffic,
+                     "kernel": "rtlynx_gemm_kernel<sparse>",
+                     "peak_note": f"2 x {peaks_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s): "
+                                  "2:4 sparse nominal ratio"},
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        line["cpu_baseline"] = oracle_sample(wl, X, W, L_A, L_B, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def kernels_per_step(R):
+    """Our kernels per sparse-mode call: norms/LoRA-down, finalize T (R > 0), compress, GEMM."""
+    return 4 if R > 0 else 3
+
+
+def kernel_rev():
+    """Hash of the GEMM kernel source, to tell whether stored ncu counters still apply."""
+    import hashlib
+    with open(os.path.join(ROOT, "activation_sparse_gemm_b200", "csrc", "gemm.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def main():
+    args = parse()
+    from activation_sparse_gemm_b200.inputs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

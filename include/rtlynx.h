@@ -1,0 +1,134 @@
+/*
+ * rtlynx.h - C ABI of the B200 (sm_100a) RT-Lynx activation-sparse linear layer.
+ *
+ * The operation (RT-Lynx summary page, paper.rainbus.top for arXiv 2605.26632,
+ * "four-step pipeline" paragraph):
+ *   step 1  X~ keeps, for every token, the 2 largest-magnitude entries of each
+ *           group of 4 consecutive input channels (ties go to the lower
+ *           channel); s = ||X||_2 / (||X~||_2 + 1e-8) per token; S(X) = s * X~.
+ *   step 2  Y = S(X) W^T + X (L_A L_B)^T, the LoRA branch fed with the dense X.
+ *   step 3  layers chosen for skipping run dense: Y = X W^T.
+ *   step 4  mask, Top-K, compression to the sparse tensor-core layout and the
+ *           sparse GEMM run in fused GPU kernels; the sparse and LoRA products
+ *           are accumulated on chip.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major bf16 (IEEE binary16-brain, little endian):
+ *       X [M, D_in], W [D_out, D_in] (nn.Linear layout), L_A [D_out, R],
+ *       L_B [R, D_in], Y [M, D_out].
+ *   - Pointers are device memory owned by the caller unless a name ends in
+ *     _host.  Inputs are only read.  Y is overwritten; it must not overlap
+ *     an input.  Every pointer must be 16-byte aligned.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream; nothing synchronizes the host
+ *     unless stated.
+ *   - Return value: an rtlynx_status.  Argument errors return before anything
+ *     is launched.
+ *   - No kernel traps.  Every device-side wait is bounded; a wait that runs
+ *     out records RTLYNX_ERR_DEVICE_TIMEOUT in a per-device error word that
+ *     rtlynx_stream_status() reads and clears.
+ */
+#ifndef RTLYNX_H
+#define RTLYNX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RTLYNX_MODE_SPARSE = 0,     /* Y = S(X) W^T + X (L_A L_B)^T  (steps 1-2) */
+    RTLYNX_MODE_DENSE_SKIP = 1  /* Y = X W^T                     (step 3)    */
+} rtlynx_mode;
+
+typedef enum {
+    RTLYNX_OK = 0,
+    RTLYNX_ERR_INVALID_ARG = 1,    /* bad size, pointer, alignment or mode        */
+    RTLYNX_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. R > 256, not sm_100) */
+    RTLYNX_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed           */
+    RTLYNX_ERR_OOM = 4,            /* workspace allocation failed                 */
+    RTLYNX_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait ran out          */
+} rtlynx_status;
+
+/*
+ * rtlynx_linear - the fused RT-Lynx linear layer (steps 1-4).
+ *   M      tokens (> 0)            D_in   input channels, > 0, multiple of 8
+ *   D_out  output channels, > 0, multiple of 8
+ *   R      LoRA rank: 0 (no LoRA branch) or a multiple of 8 up to 256; with
+ *          R = 0, or L_A / L_B NULL, sparse mode computes Y = S(X) W^T only
+ *   mode   rtlynx_mode; DENSE_SKIP ignores L_A, L_B and R
+ * Uses a workspace cached per (device, stream), grown with cudaMalloc when a
+ * larger problem arrives (the stream is synchronized before the old buffer is
+ * freed); call once outside any stream capture for each new size.
+ */
+int rtlynx_linear(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
+                  int64_t D_in, int64_t D_out, int64_t R, int mode, void* stream);
+
+/* Workspace bytes rtlynx_linear_ws needs for these sizes (0 for DENSE_SKIP;
+ * 0 also when the arguments are invalid). */
+size_t rtlynx_workspace_size(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode);
+
+/* rtlynx_linear with a caller-owned device workspace of ws_bytes bytes
+ * (>= rtlynx_workspace_size, 256-byte aligned).  Allocates nothing except,
+ * on a device's first call, its 4-byte device error word. */
+int rtlynx_linear_ws(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
+                     int64_t D_in, int64_t D_out, int64_t R, int mode, void* workspace, size_t ws_bytes,
+                     void* stream);
+
+/* rtlynx_linear_ws that also records caller-created CUDA events (cudaEvent_t
+ * passed as void*, any may be NULL) on stream: ev_start before the first
+ * kernel, ev_mid after the sparsify prologue (right before the GEMM kernel),
+ * ev_end after the GEMM kernel.  Used to time the two phases separately. */
+int rtlynx_linear_ws_events(const void* X, const void* W, const void* L_A, const void* L_B, void* Y,
+                            int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* workspace,
+                            size_t ws_bytes, void* ev_start, void* ev_mid, void* ev_end, void* stream);
+
+/* Where the sparse-mode intermediates sit inside the workspace (byte offsets),
+ * for tests that inspect them:
+ *   vals       [M_pad, Kc_pad] bf16 kept values, rows >= M zero, Kc_pad >= D_in/2
+ *   meta       [M_pad/128, k_chunks, 2048] bytes, metadata in tensor-memory order:
+ *              for token m of a 128-token block (m0 = m%8, m1 = (m/8)%2,
+ *              m2 = m/16) and channel k of a 128-channel chunk (k0 = k%16,
+ *              k1 = (k/16)%2, k2 = k/32) the group nibble i0 | (i1<<2) sits in
+ *              the 32-bit word at byte 16*(m0 + 8*k1 + 16*m2) + 4*k2, bits
+ *              16*m1 + 4*(k0/4) ... +3
+ *   s          [M_pad] float
+ *   T          [M_pad, R_pad] bf16, X L_B^T */
+typedef struct {
+    int64_t M_pad, Kc_pad, k_chunks, R_pad;
+    size_t vals, meta, s, T, total;
+} rtlynx_ws_layout;
+int rtlynx_workspace_layout(int64_t M, int64_t D_in, int64_t D_out, int64_t R, rtlynx_ws_layout* out);
+
+/* Step 1 and the LoRA down-projection alone, written in plain layouts:
+ *   vals [M, D_in/2] bf16 (kept values in channel order), meta [M, D_in/4]
+ *   uint8 (one nibble i0 | (i1<<2) per byte), s [M] float, T [M, R] bf16.
+ * Any output pointer may be NULL.  Uses the cached workspace of rtlynx_linear. */
+int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_in, int64_t R, void* vals,
+                          void* meta, void* s, void* T, void* stream);
+
+/* End-to-end form for callers whose activations live in host memory:
+ * copies X_host (pinned for overlap) to X_dev, runs rtlynx_linear into Y_dev,
+ * copies Y_dev to Y_host.  All three steps are queued on stream; synchronize
+ * the stream before reading Y_host.  W, L_A, L_B are device pointers. */
+int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const void* L_B, void* Y_host,
+                       int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* X_dev, void* Y_dev,
+                       void* stream);
+
+/* Synchronizes stream, then returns and clears the current device's error
+ * word (RTLYNX_OK or RTLYNX_ERR_DEVICE_TIMEOUT), or RTLYNX_ERR_CUDA. */
+int rtlynx_stream_status(void* stream);
+
+/* Static text for a status code. */
+const char* rtlynx_status_string(int status);
+
+/* Frees every cached workspace and error word (synchronizes the device). */
+void rtlynx_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTLYNX_H */
