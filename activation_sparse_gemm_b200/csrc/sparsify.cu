@@ -6,8 +6,9 @@
 // Pass 1  norms_lora_down   grid (row block of 128 tokens, K-split).
 //         TMA streams 128 x 64 tiles of X (128B swizzle) and 64-wide tiles of
 //         L_B.  Four warps read each X tile from shared memory, one token per
-//         thread, and accumulate sum(x^2) and sum(x~^2) (the kept entries are the
-//         two largest magnitudes of each group; ties do not change the sum).
+//         thread, and accumulate sum(x^2) and sum(x~^2) in double from exact
+//         squares (the kept entries are the two largest magnitudes of each
+//         group; ties do not change the sum).
 //         From the SAME shared-memory tile one thread issues dense tcgen05.mma
 //         (M = 128, N = R) for the partial T.  Partial sums go to the workspace.
 // Pass 2  compress          grid (16-token slab, 256-wide K block).
@@ -47,19 +48,28 @@ __host__ __device__ inline int norm_stage_bytes(int R_pad) {
     return ((kXTileBytes + R_pad * kBK * 2 + 1023) / 1024) * 1024;
 }
 
-__device__ __forceinline__ float mag_to_float(uint32_t mag15) { return __uint_as_float(mag15 << 16); }
+__device__ __forceinline__ double mag_to_double(uint32_t mag15) {
+    return static_cast<double>(__uint_as_float(mag15 << 16));
+}
 
-// sum(x^2) and sum of the two largest squares for the group in bf16 bits (lo, hi words).
-__device__ __forceinline__ void group_energy(uint32_t w01, uint32_t w23, float& all, float& kept) {
+// Adds sum(x^2) and the sum of the two largest squares of one group (bf16
+// bits in two words) to the token's double accumulators.  A bf16 square has
+// at most 16 significant bits, so every product here is exact and the sums
+// carry double rounding only (the fp32 squares of tiny bf16 values would
+// underflow, doubles do not).
+__device__ __forceinline__ void group_energy(uint32_t w01, uint32_t w23, double& all, double& kept) {
     const uint32_t a0 = w01 & 0x7FFFu, a1 = (w01 >> 16) & 0x7FFFu;
     const uint32_t a2 = w23 & 0x7FFFu, a3 = (w23 >> 16) & 0x7FFFu;
-    const float f0 = mag_to_float(a0), f1 = mag_to_float(a1), f2 = mag_to_float(a2), f3 = mag_to_float(a3);
-    all += (f0 * f0 + f1 * f1) + (f2 * f2 + f3 * f3);
     const uint32_t h01 = max(a0, a1), l01 = min(a0, a1), h23 = max(a2, a3), l23 = min(a2, a3);
-    const uint32_t t1 = max(h01, h23);
-    const uint32_t t2 = max(min(h01, h23), max(l01, l23));
-    const float g1 = mag_to_float(t1), g2 = mag_to_float(t2);
-    kept += g1 * g1 + g2 * g2;
+    const uint32_t t1 = max(h01, h23);                        // largest magnitude
+    const uint32_t t2 = max(min(h01, h23), max(l01, l23));    // second largest
+    const uint32_t u1 = min(max(l01, l23), min(h01, h23));    // third
+    const uint32_t u2 = min(l01, l23);                        // smallest
+    const double d1 = mag_to_double(t1), d2 = mag_to_double(t2);
+    const double d3 = mag_to_double(u1), d4 = mag_to_double(u2);
+    const double k = fma(d2, d2, d1 * d1);
+    kept += k;
+    all += fma(d4, d4, fma(d3, d3, k));
 }
 
 template <bool LORA>
@@ -163,15 +173,12 @@ __global__ void __launch_bounds__(kNormThreads, 1)
         for (int i = 0; i < ntiles; ++i) {
             if (!mbar_wait(&full[stage], phase, err)) break;
             const uint8_t* row = smem + stage * stage_bytes + r * 128;
-            float all = 0.f, kept = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
-                group_energy(v.x, v.y, all, kept);
-                group_energy(v.z, v.w, all, kept);
+                group_energy(v.x, v.y, nx, nt);
+                group_energy(v.z, v.w, nx, nt);
             }
-            nx += static_cast<double>(all);
-            nt += static_cast<double>(kept);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             ++consumed;

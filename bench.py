@@ -108,7 +108,9 @@ class ClockSampler:
             return
         try:
             mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-            reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            get = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            reasons = get(self.h)
             self.samples.append((mhz, reasons))
         except Exception:  # noqa: BLE001
             pass
