@@ -98,15 +98,16 @@ int validate(const void* X, const void* W, const void* L_A, const void* L_B, con
 
 }  // namespace
 
-int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                        CUtensorMapSwizzle swizzle) {
+int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle) {
+    (void)elem_bytes;
     if (!g_encode) return cudaErrorInitializationError;
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_stride_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+    CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
@@ -118,7 +119,7 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
     d.K = K;
     d.N = N;
     d.R = R;
-    d.M_pad = (M + kBM - 1) / kBM * kBM;
+    d.M_pad = (M + 2 * kBM - 1) / (2 * kBM) * (2 * kBM);
     d.m_blocks = d.M_pad / kBM;
     d.k_tiles = (K + kBK - 1) / kBK;
     d.k_chunks = (K + kChunkK - 1) / kChunkK;

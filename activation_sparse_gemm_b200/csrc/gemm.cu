@@ -1,81 +1,105 @@
-// Persistent tcgen05 GEMM for the RT-Lynx linear layer on sm_100a.
+// Persistent CTA-pair tcgen05 GEMM for the RT-Lynx linear layer on sm_100a.
 //
 //   sparse mode:      Y = S(X) W^T + T L_A^T      (RT-Lynx summary page, four-step
 //                     pipeline paragraph: step 2 gives Y = Y_s + Y_r; step 4 asks
 //                     for Y_s and Y_r to be summed on chip)
 //   dense-skip mode:  Y = X W^T                   (step 3, Selective Layer Skipping)
 //
-// One CTA per SM walks output tiles of 128 x 256.  Warp roles:
-//   warp 0      TMA producer: A tile (compressed S(X) or dense X), W tile and, in
-//               sparse mode, one 2 KB metadata chunk every second stage; then
-//               the LoRA stages (T tile and L_A tile).
-//   warp 1      TMEM owner and single-thread MMA issuer.  Sparse stages issue
-//               tcgen05.mma.sp (K = 32 logical per instruction) with the
-//               metadata copied into tensor memory by tcgen05.cp; the LoRA
-//               stages issue dense tcgen05.mma into the SAME accumulator, so
-//               T L_A^T never exists outside tensor memory.
-//   warps 2-5   epilogue: tcgen05.ld, round to bf16, 16-byte stores.
+// A cluster of two CTAs on neighbouring SMs computes one 256 x BN output tile
+// with cta_group::2 MMAs: each CTA holds 128 rows of A and BN/2 rows of W in
+// its own shared memory and 128 rows x BN columns of the f32 accumulator in
+// its own tensor memory, so each SM streams only half of the W tile.
 //
-// Shared memory per stage (1024-byte aligned):
-//   A  sparse: 128 rows x 32 kept values (64 B rows, 64B swizzle)  8 KB
-//      dense:  128 rows x 64 values      (128 B rows, 128B swizzle) 16 KB
-//   B  256 rows of W x 64 values (128B swizzle)                    32 KB
+// Warp roles in each CTA:
+//   warp 0      TMA producer.  Both CTAs load their halves; the completion of
+//               both is counted on the leader CTA's "full" barrier.  Sparse
+//               stages carry the compressed S(X) tile, the W tile and, every
+//               second stage, one 2 KB metadata chunk; then come the LoRA
+//               stages (T tile and L_A tile).
+//   warp 1      tensor-memory owner; in the leader CTA one thread issues every
+//               MMA of the pair: tcgen05.mma.sp (K = 32 logical per instruction)
+//               with the metadata moved into tensor memory by tcgen05.cp, and
+//               dense tcgen05.mma for the LoRA stages into the SAME accumulator,
+//               so T L_A^T never leaves the chip.  Its commits arrive on the
+//               barriers of both CTAs.
+//   warps 2-5   epilogue: tcgen05.ld, round to bf16, swizzled staging in shared
+//               memory, TMA store (clips the ragged M and N edges).
+// The accumulator is double-buffered in tensor memory, so the epilogue of one
+// tile overlaps the main loop of the next.
+//
+// Shared memory per CTA and stage (1024-byte aligned):
+//   A  sparse: 128 rows x 32 kept values (64 B rows, 64B swizzle)    8 KB
+//      dense:  128 rows x 64 values      (128 B rows, 128B swizzle)  16 KB
+//   B  BN/2 rows of W x 64 values (128B swizzle)                     BN*64 B
 //   E  metadata chunk, 128 lanes x 16 B, no swizzle                  2 KB (sparse)
-// LoRA stages reuse the slots: T 128 x 32 (64B swizzle) in A, L_A 256 x 32
+// LoRA stages reuse the slots: T 128 x 32 (64B swizzle) in A, L_A BN/2 x 32
 // (64B swizzle) in B.
 //
-// Tensor memory: columns [0, 256) hold the f32 accumulator (lane = tile row),
-// columns [256, 260) the metadata of the current 128-wide K chunk.
+// Tensor memory (per CTA, 512 columns): accumulators at [0, BN) and
+// [BN, 2 BN); metadata of the current 128-wide K chunk at [2 BN, 2 BN + 4).
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace rtlynx {
 
-template <bool SPARSE>
-struct GemmShape {
+constexpr int kPairThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kEpiBufBytes = 32 * 64;  // one warp's 32 rows x 32 bf16 columns
+
+template <bool SPARSE, int BN>
+struct PairShape {
+    static constexpr int BN_HALF = BN / 2;
     static constexpr int A_BYTES = SPARSE ? kBM * (kBK / 2) * 2 : kBM * kBK * 2;
-    static constexpr int B_BYTES = kBN * kBK * 2;
+    static constexpr int B_BYTES = BN_HALF * kBK * 2;
     static constexpr int E_BYTES = SPARSE ? kChunkBytes : 0;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
-    static constexpr int STAGES = 4;
+    static constexpr int STAGES = SPARSE ? 8 : 7;
     static constexpr int LORA_A_BYTES = kBM * 32 * 2;
-    static constexpr int LORA_B_BYTES = kBN * 32 * 2;
-    static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-    static_assert(LORA_A_BYTES <= A_BYTES || !SPARSE, "T tile must fit the A slot");
-    static_assert(LORA_B_BYTES <= B_BYTES, "L_A tile must fit the B slot");
+    static constexpr int LORA_B_BYTES = BN_HALF * 32 * 2;
+    static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;
+    static constexpr int BAR_BYTES = 1024;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+    static_assert(BN % 32 == 0 && BN >= 64 && 2 * BN + 4 <= 512, "two accumulators and the metadata must fit");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
+    static_assert(LORA_A_BYTES <= A_BYTES && LORA_B_BYTES <= B_BYTES, "LoRA tiles must fit the operand slots");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-struct GemmArgs {
+struct PairArgs {
     int M, N;
-    int m_blocks, n_blocks, k_tiles, lora_tiles, k_chunks;
-    const uint8_t* meta;
-    __nv_bfloat16* Y;
-    int64_t ldy;
+    int m_pairs, n_tiles, k_tiles, lora_tiles, k_chunks;
     int* err;
 };
 
-constexpr int kGemmThreads = 192;
-constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* err) {
+    uint32_t ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err) ? 1u : 0u;
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
 
-template <bool SPARSE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    rtlynx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmLA,
-                       const GemmArgs args) {
-    using G = GemmShape<SPARSE>;
+template <bool SPARSE, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    rtlynx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmLA,
+                            const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+                            const PairArgs args) {
+    using G = PairShape<SPARSE, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES);
+    uint8_t* epi = smem + G::STAGES * G::STAGE_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(epi + G::EPI_BYTES);
     uint64_t* empty = full + G::STAGES;
-    uint64_t* acc_full = empty + G::STAGES;
-    uint64_t* acc_empty = acc_full + 1;
-    uint64_t* done_bar = acc_empty + 1;
+    uint64_t* acc_full = empty + G::STAGES;   // [2]
+    uint64_t* acc_empty = acc_full + 2;       // [2], used in the leader only
+    uint64_t* done_bar = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done_bar + 1);
-    int* consumed_holder = reinterpret_cast<int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
     int* err = args.err;
 
     if (threadIdx.x == 0) {
@@ -83,41 +107,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA of the pair
+        }
         mbar_init(done_bar, 1);
-        *consumed_holder = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        prefetch_tmap(&tmY);
+        if (SPARSE) prefetch_tmap(&tmE);
         if (args.lora_tiles > 0) {
             prefetch_tmap(&tmT);
             prefetch_tmap(&tmLA);
         }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    const uint32_t tmem_acc = tmem_base;
-    const uint32_t tmem_meta = tmem_base + 256;
+    const uint32_t tmem_meta = tmem_base + 2 * BN;
 
-    const int num_tiles = args.m_blocks * args.n_blocks;
+    const int num_tiles = args.m_pairs * args.n_tiles;
     const int total_k = args.k_tiles + args.lora_tiles;
-    int issued = 0;
 
     if (warp == 0) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int mb = tile % args.m_blocks;
-                const int nb = tile / args.m_blocks;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int mp = tile % args.m_pairs;
+                const int nt = tile / args.m_pairs;
+                const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM;
+                const int col0 = nt * BN + static_cast<int>(rank) * G::BN_HALF;
                 for (int kt = 0; kt < total_k; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, err)) {
                         ok = false;
@@ -126,45 +153,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint8_t* sA = smem + stage * G::STAGE_BYTES;
                     uint8_t* sB = sA + G::A_BYTES;
                     uint8_t* sE = sB + G::B_BYTES;
+                    const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
                     if (kt < args.k_tiles) {
                         const bool with_meta = SPARSE && ((kt & 1) == 0);
-                        mbar_arrive_expect_tx(&full[stage], G::A_BYTES + G::B_BYTES + (with_meta ? G::E_BYTES : 0));
-                        tma_load_2d(sA, &tmA, &full[stage], kt * (SPARSE ? kBK / 2 : kBK), mb * kBM);
-                        tma_load_2d(sB, &tmB, &full[stage], kt * kBK, nb * kBN);
+                        if (leader)
+                            mbar_arrive_expect_tx(&full[stage],
+                                                  2u * (G::A_BYTES + G::B_BYTES + (with_meta ? G::E_BYTES : 0)));
+                        tma_load_2d_pair(sA, &tmA, fbar, kt * (SPARSE ? kBK / 2 : kBK), row0);
+                        tma_load_2d_pair(sB, &tmB, fbar, kt * kBK, col0);
                         if (with_meta) {
-                            const uint8_t* src =
-                                args.meta + (static_cast<size_t>(mb) * args.k_chunks + (kt >> 1)) * kChunkBytes;
-                            bulk_load(sE, src, kChunkBytes, &full[stage]);
+                            const int chunk = (row0 / kBM) * args.k_chunks + (kt >> 1);
+                            tma_load_2d_pair(sE, &tmE, fbar, 0, chunk * 4);
                         }
                     } else {
                         const int j = kt - args.k_tiles;
-                        mbar_arrive_expect_tx(&full[stage], G::LORA_A_BYTES + G::LORA_B_BYTES);
-                        tma_load_2d(sA, &tmT, &full[stage], j * 32, mb * kBM);
-                        tma_load_2d(sB, &tmLA, &full[stage], j * 32, nb * kBN);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2u * (G::LORA_A_BYTES + G::LORA_B_BYTES));
+                        tma_load_2d_pair(sA, &tmT, fbar, j * 32, row0);
+                        tma_load_2d_pair(sB, &tmLA, fbar, j * 32, col0);
                     }
-                    ++issued;
                     if (++stage == G::STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
+            // Wait until the leader's MMAs have released every stage this CTA
+            // filled, so no commit arrival is still on its way to this CTA.
+            for (int i = 0; i < G::STAGES && ok; ++i) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, err)) break;
+                if (++stage == G::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc_main = make_idesc_bf16(kBM, kBN, SPARSE);
-            const uint32_t idesc_dense = make_idesc_bf16(kBM, kBN, false);
+        if (leader && lane == 0) {
+            const uint32_t idesc_main = make_idesc_bf16(2 * kBM, BN, SPARSE);
+            const uint32_t idesc_dense = make_idesc_bf16(2 * kBM, BN, false);
             int stage = 0;
             uint32_t phase = 0;
-            int consumed = 0;
             int local = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                if (!mbar_wait(acc_empty, (local & 1) ^ 1u, err)) {
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+                const int buf = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1);
+                if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, err)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
                 for (int kt = 0; kt < total_k; ++kt) {
                     if (!mbar_wait(&full[stage], phase, err)) {
                         ok = false;
@@ -176,20 +215,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t sE = sB + G::B_BYTES;
                     if (kt < args.k_tiles) {
                         if constexpr (SPARSE) {
-                            if ((kt & 1) == 0) tmem_cp_128x128b(tmem_meta, make_sdesc(sE, 128, 128, kSwNone));
+                            if ((kt & 1) == 0) tmem_cp_128x128b_pair(tmem_meta, make_sdesc(sE, 128, 128, kSwNone));
 #pragma unroll
                             for (int j = 0; j < 2; ++j) {
                                 const uint64_t a = make_sdesc(sA + j * 32, 16, 512, kSw64);
                                 const uint64_t b = make_sdesc(sB + j * 64, 16, 1024, kSw128);
                                 const uint32_t e = tmem_meta + static_cast<uint32_t>((kt & 1) * 2 + j);
-                                mma_sp_f16(tmem_acc, a, b, e & ~1u, idesc_main | (e & 1u), (kt | j) != 0);
+                                mma_sp_f16_pair(d, a, b, e & ~1u, idesc_main | (e & 1u), (kt | j) != 0);
                             }
                         } else {
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const uint64_t a = make_sdesc(sA + j * 32, 16, 1024, kSw128);
                                 const uint64_t b = make_sdesc(sB + j * 32, 16, 1024, kSw128);
-                                mma_f16(tmem_acc, a, b, idesc_main, (kt | j) != 0);
+                                mma_f16_pair(d, a, b, idesc_main, (kt | j) != 0);
                             }
                         }
                     } else {
@@ -197,123 +236,151 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int j = 0; j < 2; ++j) {
                             const uint64_t a = make_sdesc(sA + j * 32, 16, 512, kSw64);
                             const uint64_t b = make_sdesc(sB + j * 32, 16, 512, kSw64);
-                            mma_f16(tmem_acc, a, b, idesc_dense, 1u);
+                            mma_f16_pair(d, a, b, idesc_dense, 1u);
                         }
                     }
-                    tc_commit(&empty[stage]);
-                    ++consumed;
+                    tc_commit_pair_mc(&empty[stage], 0x3);
                     if (++stage == G::STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
+                tc_commit_pair_mc(&acc_full[buf], 0x3);
             }
-            // Every MMA this thread issued has finished before tensor memory is freed.
-            tc_commit(done_bar);
+            // Every MMA of the pair has finished before tensor memory is freed.
+            tc_commit_pair_mc(done_bar, 0x1);
             mbar_wait(done_bar, 0, nullptr);
-            *consumed_holder = consumed;
         }
     } else {
-        const int quad = warp & 3;                 // warps 2..5 own TMEM lane quadrants 2,3,0,1
-        const int row_in_tile = quad * 32 + lane;
+        const int quad = warp & 3;  // warps 2..5 own tensor-memory lane quadrants 2,3,0,1
         const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+        uint8_t* stage_buf = epi + (warp - 2) * 2 * kEpiBufBytes;
+        int sbuf = 0;
         int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            if (!mbar_wait(acc_full, local & 1, err)) break;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
+            const int buf = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1);
+            if (!warp_wait(&acc_full[buf], use & 1u, err)) break;
             tc_fence_after();
-            const int mb = tile % args.m_blocks;
-            const int nb = tile / args.m_blocks;
-            const int64_t m = static_cast<int64_t>(mb) * kBM + row_in_tile;
-            const int n0 = nb * kBN;
+            const int mp = tile % args.m_pairs;
+            const int nt = tile / args.m_pairs;
+            const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM + quad * 32;
+            const int col0 = nt * BN;
+            const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN) + lane_addr;
 #pragma unroll 1
-            for (int c = 0; c < kBN; c += 32) {
+            for (int c = 0; c < BN; c += 32) {
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_acc + lane_addr + static_cast<uint32_t>(c), r);
+                tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), r);
                 tmem_ld_wait();
-                if (m < args.M) {
-                    __nv_bfloat16* yrow = args.Y + m * args.ldy + n0 + c;
+                uint8_t* sb = stage_buf + sbuf * kEpiBufBytes;
+                if (lane == 0) bulk_wait_group_read<1>();  // the store that last used sb has read it
+                __syncwarp();
+                uint8_t* row = sb + lane * 64;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (n0 + c + v * 8 < args.N) {
-                            uint4 pk;
-                            pk.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-                            pk.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-                            pk.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-                            pk.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-                            *reinterpret_cast<uint4*>(yrow + v * 8) = pk;
-                        }
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                    pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                    pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                    pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                    *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) = pk;
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, sb, col0 + c, row0);
+                    bulk_commit_group();
+                }
+                sbuf ^= 1;
             }
             tc_fence_before();
-            mbar_arrive(acc_empty);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
         }
+        if (lane == 0) bulk_wait_all();
     }
 
-    __syncthreads();
-    if (warp == 0 && lane == 0) {
-        // After an abort, wait for copies still in flight into this CTA's shared memory.
-        for (int q = *consumed_holder; q < issued; ++q)
-            mbar_wait(&full[q % G::STAGES], (q / G::STAGES) & 1, nullptr);
+    // After an abort, give copies still in flight time to land before the
+    // shared memory they target is released.
+    if (error_seen(err)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
     }
+    tc_fence_before();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
-template <bool SPARSE>
-static int launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmT,
-                            const CUtensorMap& tmLA, const GemmArgs& args, int num_sms, cudaStream_t stream) {
-    using G = GemmShape<SPARSE>;
-    auto kernel = rtlynx_gemm_kernel<SPARSE>;
+template <bool SPARSE, int BN>
+static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmT,
+                       const CUtensorMap& tmLA, const CUtensorMap& tmE, const CUtensorMap& tmY, const PairArgs& args,
+                       int num_sms, cudaStream_t stream) {
+    using G = PairShape<SPARSE, BN>;
+    auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const int tiles = args.m_blocks * args.n_blocks;
-    const int grid = tiles < num_sms ? tiles : num_sms;
-    kernel<<<grid, kGemmThreads, G::SMEM_BYTES, stream>>>(tmA, tmB, tmT, tmLA, args);
+    const int tiles = args.m_pairs * args.n_tiles;
+    const int max_pairs = num_sms / 2;
+    const int pairs = tiles < max_pairs ? tiles : max_pairs;
+    kernel<<<2 * pairs, kPairThreads, G::SMEM_BYTES, stream>>>(tmA, tmB, tmT, tmLA, tmE, tmY, args);
     return cudaGetLastError();
 }
 
+constexpr int kPairBN = 192;
+
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream) {
-    CUtensorMap tmA, tmB, tmT, tmLA;
+    constexpr int BN = kPairBN;
+    CUtensorMap tmA, tmB, tmT, tmLA, tmE, tmY;
     int rc;
     if (sparse) {
-        rc = encode_tmap_bf16_2d(&tmA, ws.vals, d.Kc_pad, d.M_pad, d.Kc_pad * 2, kBK / 2, kBM,
-                                 CU_TENSOR_MAP_SWIZZLE_64B);
+        rc = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.vals, d.Kc_pad, d.M_pad, d.Kc_pad * 2,
+                            kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_64B);
+        if (rc) return rc;
+        // metadata chunks viewed as rows of 256 16-bit words, four rows per chunk
+        rc = encode_tmap_2d(&tmE, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, ws.meta, 256, d.m_blocks * d.k_chunks * 4, 512,
+                            256, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc) return rc;
     } else {
-        rc = encode_tmap_bf16_2d(&tmA, A, d.K, d.M, d.K * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+        rc = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, d.K, d.M, d.K * 2, kBK, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+        tmE = tmA;
     }
+    rc = encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, d.K, d.N, d.K * 2, kBK, BN / 2,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
-    rc = encode_tmap_bf16_2d(&tmB, W, d.K, d.N, d.K * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    rc = encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d.N, d.M, d.N * 2, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
     const bool lora = sparse && d.R > 0 && L_A != nullptr;
     if (lora) {
-        rc = encode_tmap_bf16_2d(&tmT, ws.T, d.R_pad, d.M_pad, d.R_pad * 2, 32, kBM, CU_TENSOR_MAP_SWIZZLE_64B);
+        rc = encode_tmap_2d(&tmT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.T, d.R_pad, d.M_pad, d.R_pad * 2, 32, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_64B);
         if (rc) return rc;
-        rc = encode_tmap_bf16_2d(&tmLA, L_A, d.R, d.N, d.R * 2, 32, kBN, CU_TENSOR_MAP_SWIZZLE_64B);
+        rc = encode_tmap_2d(&tmLA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L_A, d.R, d.N, d.R * 2, 32, BN / 2,
+                            CU_TENSOR_MAP_SWIZZLE_64B);
         if (rc) return rc;
     } else {
         tmT = tmA;
         tmLA = tmB;
     }
-    GemmArgs args;
+    PairArgs args;
     args.M = static_cast<int>(d.M);
     args.N = static_cast<int>(d.N);
-    args.m_blocks = static_cast<int>(sparse ? d.m_blocks : (d.M + kBM - 1) / kBM);
-    args.n_blocks = static_cast<int>((d.N + kBN - 1) / kBN);
+    args.m_pairs = static_cast<int>((d.M + 2 * kBM - 1) / (2 * kBM));
+    args.n_tiles = static_cast<int>((d.N + BN - 1) / BN);
     args.k_tiles = static_cast<int>(d.k_tiles);
     args.lora_tiles = lora ? static_cast<int>(d.R_pad / 32) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
-    args.meta = ws.meta;
-    args.Y = static_cast<__nv_bfloat16*>(Y);
-    args.ldy = d.N;
     args.err = err;
-    return sparse ? launch_gemm_impl<true>(tmA, tmB, tmT, tmLA, args, num_sms, stream)
-                  : launch_gemm_impl<false>(tmA, tmB, tmT, tmLA, args, num_sms, stream);
+    return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, args, num_sms, stream)
+                  : launch_pair<false, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, args, num_sms, stream);
 }
 
 }  // namespace rtlynx

@@ -18,7 +18,7 @@ constexpr int kChunkBytes = 2048; // 128 lanes x 16 bytes of metadata per chunk
 // Sizes derived from one problem.
 struct Dims {
     int64_t M, K, N, R;
-    int64_t M_pad;        // M rounded up to kBM
+    int64_t M_pad;        // M rounded up to 2 * kBM (one CTA pair of the GEMM)
     int64_t m_blocks;     // M_pad / kBM
     int64_t k_tiles;      // ceil(K / kBK)
     int64_t k_chunks;     // ceil(K / kChunkK)
@@ -45,9 +45,15 @@ struct Workspace {
 };
 
 // Tensor-map encoding through the driver entry point (no libcuda link needed).
-int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                        CUtensorMapSwizzle swizzle);
+int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle);
+inline int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                               CUtensorMapSwizzle swizzle) {
+    return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, row_stride_bytes, box_inner,
+                          box_outer, swizzle);
+}
 
 // Launchers; each returns a cudaError_t value (0 on success).
 int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
