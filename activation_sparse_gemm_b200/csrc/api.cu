@@ -123,8 +123,8 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
     d.m_blocks = d.M_pad / kBM;
     d.k_tiles = (K + kBK - 1) / kBK;
     d.k_chunks = (K + kChunkK - 1) / kChunkK;
-    d.Kc_pad = d.k_tiles * (kBK / 2);
-    d.R_pad = R > 0 ? (R + 31) / 32 * 32 : 0;
+    d.Kc_pad = d.k_chunks * (kChunkK / 2);
+    d.R_pad = R > 0 ? (R + 63) / 64 * 64 : 0;
     // Enough CTAs in the norm / LoRA-down pass to cover the GPU about twice,
     // every split holding at least one K tile.
     int64_t target = 2 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148);

@@ -27,13 +27,17 @@
 // The accumulator is double-buffered in tensor memory, so the epilogue of one
 // tile overlaps the main loop of the next.
 //
-// Shared memory per CTA and stage (1024-byte aligned):
-//   A  sparse: 128 rows x 32 kept values (64 B rows, 64B swizzle)    8 KB
-//      dense:  128 rows x 64 values      (128 B rows, 128B swizzle)  16 KB
-//   B  BN/2 rows of W x 64 values (128B swizzle)                     BN*64 B
-//   E  metadata chunk, 128 lanes x 16 B, no swizzle                  2 KB (sparse)
-// LoRA stages reuse the slots: T 128 x 32 (64B swizzle) in A, L_A BN/2 x 32
-// (64B swizzle) in B.
+// Shared memory per CTA and stage (1024-byte aligned, 128B swizzle):
+//   sparse stage, 128 logical K:
+//     A  128 rows x 64 kept values                                  16 KB
+//     B  BN/2 rows of W x 128 values, two 64-wide column blocks     BN*128 B
+//     E  the metadata chunk of these 128 K, 128 lanes x 16 B         2 KB
+//   dense stage, 64 logical K:  A 128 x 64 (16 KB), B BN/2 x 64 (BN*64 B)
+// LoRA stages reuse the slots: T 128 x 64 in A, L_A BN/2 x 64 in B, four
+// dense K = 16 MMAs per stage.
+// The single MMA-issuing thread is latency bound on its own instruction
+// chain, so its loop only adds precomputed offsets to precomputed
+// descriptors and every stage carries four MMAs per barrier round trip.
 //
 // Tensor memory (per CTA, 512 columns): accumulators at [0, BN) and
 // [BN, 2 BN); metadata of the current 128-wide K chunk at [2 BN, 2 BN + 4).
@@ -49,25 +53,30 @@ constexpr int kEpiBufBytes = 32 * 64;  // one warp's 32 rows x 32 bf16 columns
 template <bool SPARSE, int BN>
 struct PairShape {
     static constexpr int BN_HALF = BN / 2;
-    static constexpr int A_BYTES = SPARSE ? kBM * (kBK / 2) * 2 : kBM * kBK * 2;
-    static constexpr int B_BYTES = BN_HALF * kBK * 2;
+    static constexpr int BK = SPARSE ? 128 : 64;                 // logical K per stage
+    static constexpr int A_BYTES = kBM * 64 * 2;                  // 128 rows x 128 B
+    static constexpr int B_ATOM_BYTES = BN_HALF * 64 * 2;        // BN/2 rows x 128 B
+    static constexpr int B_BYTES = (BK / 64) * B_ATOM_BYTES;
     static constexpr int E_BYTES = SPARSE ? kChunkBytes : 0;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
-    static constexpr int STAGES = SPARSE ? 8 : 7;
-    static constexpr int LORA_A_BYTES = kBM * 32 * 2;
-    static constexpr int LORA_B_BYTES = BN_HALF * 32 * 2;
+    static constexpr int STAGES = SPARSE ? 4 : 7;
+    static constexpr int LORA_A_BYTES = kBM * 64 * 2;
+    static constexpr int LORA_B_BYTES = BN_HALF * 64 * 2;
     static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
     static_assert(BN % 32 == 0 && BN >= 64 && 2 * BN + 4 <= 512, "two accumulators and the metadata must fit");
-    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
+    static_assert(B_ATOM_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
     static_assert(LORA_A_BYTES <= A_BYTES && LORA_B_BYTES <= B_BYTES, "LoRA tiles must fit the operand slots");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct PairArgs {
     int M, N;
-    int m_pairs, n_tiles, k_tiles, lora_tiles, k_chunks;
+    int m_pairs, n_tiles;
+    int k_stages;      // main-loop stages per tile (128-wide K chunks when sparse, 64-wide when dense)
+    int lora_stages;   // 64-wide LoRA stages per tile
+    int k_chunks;      // metadata chunks per 128-row block
     int* err;
 };
 
@@ -117,7 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmY);
         if (SPARSE) prefetch_tmap(&tmE);
-        if (args.lora_tiles > 0) {
+        if (args.lora_stages > 0) {
             prefetch_tmap(&tmT);
             prefetch_tmap(&tmLA);
         }
@@ -133,10 +142,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_meta = tmem_base + 2 * BN;
 
     const int num_tiles = args.m_pairs * args.n_tiles;
-    const int total_k = args.k_tiles + args.lora_tiles;
+    const int total_k = args.k_stages + args.lora_stages;
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -145,6 +155,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 const int nt = tile / args.m_pairs;
                 const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM;
                 const int col0 = nt * BN + static_cast<int>(rank) * G::BN_HALF;
+                const int chunk0 = (row0 / kBM) * args.k_chunks;
                 for (int kt = 0; kt < total_k; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, err)) {
                         ok = false;
@@ -152,24 +163,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     }
                     uint8_t* sA = smem + stage * G::STAGE_BYTES;
                     uint8_t* sB = sA + G::A_BYTES;
-                    uint8_t* sE = sB + G::B_BYTES;
-                    const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
-                    if (kt < args.k_tiles) {
-                        const bool with_meta = SPARSE && ((kt & 1) == 0);
-                        if (leader)
-                            mbar_arrive_expect_tx(&full[stage],
-                                                  2u * (G::A_BYTES + G::B_BYTES + (with_meta ? G::E_BYTES : 0)));
-                        tma_load_2d_pair(sA, &tmA, fbar, kt * (SPARSE ? kBK / 2 : kBK), row0);
-                        tma_load_2d_pair(sB, &tmB, fbar, kt * kBK, col0);
-                        if (with_meta) {
-                            const int chunk = (row0 / kBM) * args.k_chunks + (kt >> 1);
-                            tma_load_2d_pair(sE, &tmE, fbar, 0, chunk * 4);
+                    const uint32_t fbar = full0 + static_cast<uint32_t>(stage) * 8u;
+                    if (kt < args.k_stages) {
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2u * (G::A_BYTES + G::B_BYTES + G::E_BYTES));
+                        tma_load_2d_pair(sA, &tmA, fbar, kt * 64, row0);
+                        tma_load_2d_pair(sB, &tmB, fbar, kt * G::BK, col0);
+                        if constexpr (SPARSE) {
+                            tma_load_2d_pair(sB + G::B_ATOM_BYTES, &tmB, fbar, kt * G::BK + 64, col0);
+                            tma_load_2d_pair(sB + G::B_BYTES, &tmE, fbar, 0, (chunk0 + kt) * 4);
                         }
                     } else {
-                        const int j = kt - args.k_tiles;
+                        const int j = kt - args.k_stages;
                         if (leader) mbar_arrive_expect_tx(&full[stage], 2u * (G::LORA_A_BYTES + G::LORA_B_BYTES));
-                        tma_load_2d_pair(sA, &tmT, fbar, j * 32, row0);
-                        tma_load_2d_pair(sB, &tmLA, fbar, j * 32, col0);
+                        tma_load_2d_pair(sA, &tmT, fbar, j * 64, row0);
+                        tma_load_2d_pair(sB, &tmLA, fbar, j * 64, col0);
                     }
                     if (++stage == G::STAGES) {
                         stage = 0;
@@ -191,8 +198,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (leader && lane == 0) {
             const uint32_t idesc_main = make_idesc_bf16(2 * kBM, BN, SPARSE);
             const uint32_t idesc_dense = make_idesc_bf16(2 * kBM, BN, false);
+            // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the
+            // start-address field, operand offsets inside a stage likewise.
+            const uint32_t smem0 = smem_u32(smem);
+            const uint64_t descA0 = make_sdesc(smem0, 16, 1024, kSw128);
+            const uint64_t descB0 = make_sdesc(smem0 + G::A_BYTES, 16, 1024, kSw128);
+            const uint64_t descE0 = make_sdesc(smem0 + G::A_BYTES + G::B_BYTES, 128, 128, kSwNone);
+            constexpr uint64_t kStageStep = G::STAGE_BYTES >> 4;
+            constexpr uint64_t kAtomStep = G::B_ATOM_BYTES >> 4;
+            // metadata column of sparse MMA j: (tmem_meta + j) with bit 0 moved to the selector
+            const uint32_t e01 = tmem_meta & ~1u, e23 = (tmem_meta + 2u) & ~1u;
+            const uint32_t id0 = idesc_main | (tmem_meta & 1u), id1 = idesc_main | ((tmem_meta + 1u) & 1u);
             int stage = 0;
             uint32_t phase = 0;
+            uint64_t off = 0;  // stage offset in 16-byte units
             int local = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
@@ -210,38 +229,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sA = smem_u32(smem + stage * G::STAGE_BYTES);
-                    const uint32_t sB = sA + G::A_BYTES;
-                    const uint32_t sE = sB + G::B_BYTES;
-                    if (kt < args.k_tiles) {
+                    const uint64_t a = descA0 + off;
+                    const uint64_t b = descB0 + off;
+                    if (kt < args.k_stages) {
+                        const uint32_t acc = kt != 0;
                         if constexpr (SPARSE) {
-                            if ((kt & 1) == 0) tmem_cp_128x128b_pair(tmem_meta, make_sdesc(sE, 128, 128, kSwNone));
-#pragma unroll
-                            for (int j = 0; j < 2; ++j) {
-                                const uint64_t a = make_sdesc(sA + j * 32, 16, 512, kSw64);
-                                const uint64_t b = make_sdesc(sB + j * 64, 16, 1024, kSw128);
-                                const uint32_t e = tmem_meta + static_cast<uint32_t>((kt & 1) * 2 + j);
-                                mma_sp_f16_pair(d, a, b, e & ~1u, idesc_main | (e & 1u), (kt | j) != 0);
-                            }
+                            tmem_cp_128x128b_pair(tmem_meta, descE0 + off);
+                            mma_sp_f16_pair(d, a, b, e01, id0, acc);
+                            mma_sp_f16_pair(d, a + 2, b + 4, e01, id1, 1u);
+                            mma_sp_f16_pair(d, a + 4, b + kAtomStep, e23, id0, 1u);
+                            mma_sp_f16_pair(d, a + 6, b + kAtomStep + 4, e23, id1, 1u);
                         } else {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const uint64_t a = make_sdesc(sA + j * 32, 16, 1024, kSw128);
-                                const uint64_t b = make_sdesc(sB + j * 32, 16, 1024, kSw128);
-                                mma_f16_pair(d, a, b, idesc_main, (kt | j) != 0);
-                            }
+                            mma_f16_pair(d, a, b, idesc_main, acc);
+                            mma_f16_pair(d, a + 2, b + 2, idesc_main, 1u);
+                            mma_f16_pair(d, a + 4, b + 4, idesc_main, 1u);
+                            mma_f16_pair(d, a + 6, b + 6, idesc_main, 1u);
                         }
                     } else {
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const uint64_t a = make_sdesc(sA + j * 32, 16, 512, kSw64);
-                            const uint64_t b = make_sdesc(sB + j * 32, 16, 512, kSw64);
-                            mma_f16_pair(d, a, b, idesc_dense, 1u);
-                        }
+                        mma_f16_pair(d, a, b, idesc_dense, 1u);
+                        mma_f16_pair(d, a + 2, b + 2, idesc_dense, 1u);
+                        mma_f16_pair(d, a + 4, b + 4, idesc_dense, 1u);
+                        mma_f16_pair(d, a + 6, b + 6, idesc_dense, 1u);
                     }
                     tc_commit_pair_mc(&empty[stage], 0x3);
+                    off += kStageStep;
                     if (++stage == G::STAGES) {
                         stage = 0;
+                        off = 0;
                         phase ^= 1u;
                     }
                 }
@@ -340,7 +354,7 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     int rc;
     if (sparse) {
         rc = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.vals, d.Kc_pad, d.M_pad, d.Kc_pad * 2,
-                            kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_64B);
+                            64, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
         // metadata chunks viewed as rows of 256 16-bit words, four rows per chunk
         rc = encode_tmap_2d(&tmE, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, ws.meta, 256, d.m_blocks * d.k_chunks * 4, 512,
@@ -360,11 +374,11 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     if (rc) return rc;
     const bool lora = sparse && d.R > 0 && L_A != nullptr;
     if (lora) {
-        rc = encode_tmap_2d(&tmT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.T, d.R_pad, d.M_pad, d.R_pad * 2, 32, kBM,
-                            CU_TENSOR_MAP_SWIZZLE_64B);
+        rc = encode_tmap_2d(&tmT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.T, d.R_pad, d.M_pad, d.R_pad * 2, 64, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
-        rc = encode_tmap_2d(&tmLA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L_A, d.R, d.N, d.R * 2, 32, BN / 2,
-                            CU_TENSOR_MAP_SWIZZLE_64B);
+        rc = encode_tmap_2d(&tmLA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L_A, d.R, d.N, d.R * 2, 64, BN / 2,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
     } else {
         tmT = tmA;
@@ -375,8 +389,8 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.N = static_cast<int>(d.N);
     args.m_pairs = static_cast<int>((d.M + 2 * kBM - 1) / (2 * kBM));
     args.n_tiles = static_cast<int>((d.N + BN - 1) / BN);
-    args.k_tiles = static_cast<int>(d.k_tiles);
-    args.lora_tiles = lora ? static_cast<int>(d.R_pad / 32) : 0;
+    args.k_stages = static_cast<int>(sparse ? d.k_chunks : d.k_tiles);
+    args.lora_stages = lora ? static_cast<int>(d.R_pad / 64) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
     args.err = err;
     return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, args, num_sms, stream)

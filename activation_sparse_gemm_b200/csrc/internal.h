@@ -22,8 +22,8 @@ struct Dims {
     int64_t m_blocks;     // M_pad / kBM
     int64_t k_tiles;      // ceil(K / kBK)
     int64_t k_chunks;     // ceil(K / kChunkK)
-    int64_t Kc_pad;       // compressed row length in elements = k_tiles * kBK / 2
-    int64_t R_pad;        // R rounded up to 32 (0 when R == 0)
+    int64_t Kc_pad;       // compressed row length in elements = k_chunks * kChunkK / 2
+    int64_t R_pad;        // R rounded up to 64 (0 when R == 0)
     int64_t nsplit;       // K-splits of the norm / LoRA-down pass
 };
 
