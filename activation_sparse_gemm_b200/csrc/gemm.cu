@@ -39,6 +39,9 @@
 // chain, so its loop only adds precomputed offsets to precomputed
 // descriptors and every stage carries four MMAs per barrier round trip.
 //
+// BN = 240 keeps two accumulators and the metadata inside 512 columns; the
+// epilogue writes it as seven 32-column chunks and one 16-column chunk.
+//
 // Tensor memory (per CTA, 512 columns): accumulators at [0, BN) and
 // [BN, 2 BN); metadata of the current 128-wide K chunk at [2 BN, 2 BN + 4).
 #include "internal.h"
@@ -59,13 +62,13 @@ struct PairShape {
     static constexpr int B_BYTES = (BK / 64) * B_ATOM_BYTES;
     static constexpr int E_BYTES = SPARSE ? kChunkBytes : 0;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
-    static constexpr int STAGES = SPARSE ? 4 : 7;
+    static constexpr int STAGES = SPARSE ? 4 : 6;
     static constexpr int LORA_A_BYTES = kBM * 64 * 2;
     static constexpr int LORA_B_BYTES = BN_HALF * 64 * 2;
     static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-    static_assert(BN % 32 == 0 && BN >= 64 && 2 * BN + 4 <= 512, "two accumulators and the metadata must fit");
+    static_assert(BN % 16 == 0 && BN >= 64 && 2 * BN + 4 <= 512, "two accumulators and the metadata must fit");
     static_assert(B_ATOM_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
     static_assert(LORA_A_BYTES <= A_BYTES && LORA_B_BYTES <= B_BYTES, "LoRA tiles must fit the operand slots");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -91,7 +94,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     rtlynx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmLA,
                             const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-                            const PairArgs args) {
+                            const __grid_constant__ CUtensorMap tmY16, const PairArgs args) {
     using G = PairShape<SPARSE, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,6 +128,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmY);
+        if (BN % 32) prefetch_tmap(&tmY16);
         if (SPARSE) prefetch_tmap(&tmE);
         if (args.lora_stages > 0) {
             prefetch_tmap(&tmT);
@@ -284,26 +288,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN) + lane_addr;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
+                const bool half = (BN - c) < 32;  // 16-column tail chunk
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), r);
-                tmem_ld_wait();
+                if (half) {
+                    uint32_t h[16];
+                    tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), h);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) r[q] = h[q];
+                } else {
+                    tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), r);
+                    tmem_ld_wait();
+                }
                 uint8_t* sb = stage_buf + sbuf * kEpiBufBytes;
                 if (lane == 0) bulk_wait_group_read<1>();  // the store that last used sb has read it
                 __syncwarp();
-                uint8_t* row = sb + lane * 64;
+                if (!half) {
+                    // 32 rows x 64 B, 64B swizzle: 16-byte unit q of row i at q ^ ((i / 2) % 4)
+                    uint8_t* row = sb + lane * 64;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 pk;
-                    pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-                    pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-                    pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-                    pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-                    *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) = pk;
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                        pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                        pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                        pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                        *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) = pk;
+                    }
+                } else {
+                    // 32 rows x 32 B, 32B swizzle: 16-byte unit q of row i at q ^ ((i / 4) % 2)
+                    uint8_t* row = sb + lane * 32;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                        pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                        pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                        pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                        *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 2) & 1)) << 4)) = pk;
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmY, sb, col0 + c, row0);
+                    tma_store_2d(half ? &tmY16 : &tmY, sb, col0 + c, row0);
                     bulk_commit_group();
                 }
                 sbuf ^= 1;
@@ -332,8 +360,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
 template <bool SPARSE, int BN>
 static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmT,
-                       const CUtensorMap& tmLA, const CUtensorMap& tmE, const CUtensorMap& tmY, const PairArgs& args,
-                       int num_sms, cudaStream_t stream) {
+                       const CUtensorMap& tmLA, const CUtensorMap& tmE, const CUtensorMap& tmY,
+                       const CUtensorMap& tmY16, const PairArgs& args, int num_sms, cudaStream_t stream) {
     using G = PairShape<SPARSE, BN>;
     auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
@@ -341,16 +369,16 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
     const int tiles = args.m_pairs * args.n_tiles;
     const int max_pairs = num_sms / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
-    kernel<<<2 * pairs, kPairThreads, G::SMEM_BYTES, stream>>>(tmA, tmB, tmT, tmLA, tmE, tmY, args);
+    kernel<<<2 * pairs, kPairThreads, G::SMEM_BYTES, stream>>>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args);
     return cudaGetLastError();
 }
 
-constexpr int kPairBN = 192;
+constexpr int kPairBN = 240;
 
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream) {
     constexpr int BN = kPairBN;
-    CUtensorMap tmA, tmB, tmT, tmLA, tmE, tmY;
+    CUtensorMap tmA, tmB, tmT, tmLA, tmE, tmY, tmY16;
     int rc;
     if (sparse) {
         rc = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.vals, d.Kc_pad, d.M_pad, d.Kc_pad * 2,
@@ -371,6 +399,9 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     if (rc) return rc;
     rc = encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d.N, d.M, d.N * 2, 32, 32,
                         CU_TENSOR_MAP_SWIZZLE_64B);
+    if (rc) return rc;
+    rc = encode_tmap_2d(&tmY16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d.N, d.M, d.N * 2, 16, 32,
+                        CU_TENSOR_MAP_SWIZZLE_32B);
     if (rc) return rc;
     const bool lora = sparse && d.R > 0 && L_A != nullptr;
     if (lora) {
@@ -393,8 +424,8 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.lora_stages = lora ? static_cast<int>(d.R_pad / 64) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
     args.err = err;
-    return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, args, num_sms, stream)
-                  : launch_pair<false, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, args, num_sms, stream);
+    return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
+                  : launch_pair<false, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
 }
 
 }  // namespace rtlynx
