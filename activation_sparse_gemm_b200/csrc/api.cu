@@ -189,7 +189,10 @@ static int cached_workspace(int dev, cudaStream_t stream, size_t bytes, void** o
 }
 
 static int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
-                        cudaStream_t stream) {
+                        int num_sms, cudaStream_t stream) {
+    int cpc = 0;
+    const int cs = pick_cluster_split(d, num_sms, &cpc);
+    if (cs > 0) return launch_sparsify_cluster(d, cs, cpc, X, L_B, ws, err, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;
     if (launch_norms_lora_down(d, X, L_B, ws, err, stream)) return RTLYNX_ERR_CUDA;
     if (launch_compress(d, X, ws, stream)) return RTLYNX_ERR_CUDA;
     return RTLYNX_OK;
@@ -253,7 +256,7 @@ int rtlynx_linear_ws_events(const void* X, const void* W, const void* L_A, const
         return RTLYNX_ERR_INVALID_ARG;
     const Workspace ws = carve(workspace, l);
     if (!record(ev_start)) return RTLYNX_ERR_CUDA;
-    rc = run_prologue(d, X, lora ? L_B : nullptr, ws, di->err_word, stream);
+    rc = run_prologue(d, X, lora ? L_B : nullptr, ws, di->err_word, di->num_sms, stream);
     if (rc) return rc;
     if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
     if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, di->num_sms, di->err_word, stream))
@@ -304,7 +307,7 @@ int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_i
     rc = cached_workspace(dev, stream, l.total, &base);
     if (rc) return rc;
     const Workspace ws = carve(base, l);
-    rc = run_prologue(d, X, R > 0 ? L_B : nullptr, ws, di->err_word, stream);
+    rc = run_prologue(d, X, R > 0 ? L_B : nullptr, ws, di->err_word, di->num_sms, stream);
     if (rc) return rc;
     if (launch_unpack_debug(d, ws, vals, meta, s, R > 0 ? T : nullptr, stream)) return RTLYNX_ERR_CUDA;
     return RTLYNX_OK;

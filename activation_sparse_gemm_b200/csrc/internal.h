@@ -59,6 +59,11 @@ inline int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inne
 int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
                            cudaStream_t stream);
 int launch_compress(const Dims& d, const void* X, const Workspace& ws, cudaStream_t stream);
+// One-pass prologue through CTA clusters; pick_cluster_split returns the
+// cluster size (0 when the slice does not fit and the two-pass path is used).
+int pick_cluster_split(const Dims& d, int num_sms, int* chunks_per_cta);
+int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, const void* X, const void* L_B,
+                            const Workspace& ws, int* err, cudaStream_t stream);
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream);
 int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,

@@ -27,6 +27,7 @@
 // and the nibble of a group is i0 | (i1 << 2) with i0 < i1 the kept indices.
 #include "internal.h"
 #include "ptx.cuh"
+#include "sparsify_math.cuh"
 
 namespace rtlynx {
 
@@ -46,30 +47,6 @@ constexpr int kXTileBytes = kBM * kBK * 2;  // 16 KB
 
 __host__ __device__ inline int norm_stage_bytes(int R_pad) {
     return ((kXTileBytes + R_pad * kBK * 2 + 1023) / 1024) * 1024;
-}
-
-__device__ __forceinline__ double mag_to_double(uint32_t mag15) {
-    return static_cast<double>(__uint_as_float(mag15 << 16));
-}
-
-// Adds sum(x^2) and the sum of the two largest squares of one group (bf16
-// bits in two words) to the token's double accumulators.  A bf16 square has
-// at most 16 significant bits, so every product here is exact and the sums
-// carry double rounding only (the fp32 squares of tiny bf16 values would
-// underflow, doubles do not).
-__device__ __forceinline__ void group_energy(uint32_t w01, uint32_t w23, double& all, double& kept) {
-    const uint32_t a0 = w01 & 0x7FFFu, a1 = (w01 >> 16) & 0x7FFFu;
-    const uint32_t a2 = w23 & 0x7FFFu, a3 = (w23 >> 16) & 0x7FFFu;
-    const uint32_t h01 = max(a0, a1), l01 = min(a0, a1), h23 = max(a2, a3), l23 = min(a2, a3);
-    const uint32_t t1 = max(h01, h23);                        // largest magnitude
-    const uint32_t t2 = max(min(h01, h23), max(l01, l23));    // second largest
-    const uint32_t u1 = min(max(l01, l23), min(h01, h23));    // third
-    const uint32_t u2 = min(l01, l23);                        // smallest
-    const double d1 = mag_to_double(t1), d2 = mag_to_double(t2);
-    const double d3 = mag_to_double(u1), d4 = mag_to_double(u2);
-    const double k = fma(d2, d2, d1 * d1);
-    kept += k;
-    all += fma(d4, d4, fma(d3, d3, k));
 }
 
 template <bool LORA>
@@ -234,50 +211,6 @@ struct CompressArgs {
     uint8_t* meta;
     float* s_out;
 };
-
-// bf16 nearest-even of the exact product s*x (one rounding, like the definition).
-__device__ __forceinline__ uint32_t mul_round_bf16(float s, float x) {
-    const float p = __fmul_rn(s, x);
-    const float e = __fmaf_rn(s, x, -p);  // s*x - p, exact
-    const uint32_t u = __float_as_uint(p);
-    if ((u & 0xFFFFu) == 0x8000u && e != 0.0f) {
-        const uint32_t t = u & 0xFFFF0000u;
-        const bool away = (e > 0.0f) == (p > 0.0f);
-        return (away ? t + 0x10000u : t) >> 16;
-    }
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(p)));
-}
-
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
-
-// One group of four bf16 (bits packed in two words): kept indices by the
-// 2-of-4 rule (magnitude, ties to the lower index); returns the nibble and the
-// two rounded, scaled kept values packed as bf16x2.
-__device__ __forceinline__ uint32_t compress_group(uint32_t w01, uint32_t w23, float s, uint32_t& packed) {
-    const uint32_t b[4] = {w01 & 0xFFFFu, w01 >> 16, w23 & 0xFFFFu, w23 >> 16};
-    const uint32_t m[4] = {b[0] & 0x7FFFu, b[1] & 0x7FFFu, b[2] & 0x7FFFu, b[3] & 0x7FFFu};
-    int beaten[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int i = 1; i < 4; ++i) {
-#pragma unroll
-        for (int j = 0; j < i; ++j) {
-            if (m[j] >= m[i]) ++beaten[i];  // j < i wins ties
-            else ++beaten[j];
-        }
-    }
-    int i0 = -1, i1 = -1;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (beaten[i] < 2) {
-            if (i0 < 0) i0 = i;
-            else i1 = i;
-        }
-    }
-    const uint32_t v0 = mul_round_bf16(s, bf16_bits_to_float(b[i0]));
-    const uint32_t v1 = mul_round_bf16(s, bf16_bits_to_float(b[i1]));
-    packed = v0 | (v1 << 16);
-    return static_cast<uint32_t>(i0 | (i1 << 2));
-}
 
 __global__ void __launch_bounds__(256) rtlynx_compress_kernel(const uint16_t* __restrict__ X, const CompressArgs a) {
     const int warp = threadIdx.x >> 5;
