@@ -36,8 +36,8 @@ ERR_DEVICE_TIMEOUT = 5
 ABI_SYMBOLS = (
     "rtlynx_linear", "rtlynx_workspace_size", "rtlynx_linear_ws", "rtlynx_linear_ws_events",
     "rtlynx_workspace_layout",
-    "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_stream_status", "rtlynx_status_string",
-    "rtlynx_release",
+    "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_kernel_launches", "rtlynx_stream_status",
+    "rtlynx_status_string", "rtlynx_release",
 )
 
 _lib = None
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_sparsify_debug.restype = i
         L.rtlynx_linear_host.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i, p, p, p]
         L.rtlynx_linear_host.restype = i
+        L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
+        L.rtlynx_kernel_launches.restype = i
         L.rtlynx_stream_status.argtypes = [p]
         L.rtlynx_stream_status.restype = i
         L.rtlynx_status_string.argtypes = [i]
@@ -157,6 +159,10 @@ def rtlynx_linear_host(X_host, W, L_A, L_B, Y_host, M, D_in, D_out, R, mode, X_d
     return _check(lib().rtlynx_linear_host(_ptr(X_host), _ptr(W), _ptr(L_A), _ptr(L_B), _ptr(Y_host), M, D_in,
                                            D_out, R, mode, _ptr(X_dev), _ptr(Y_dev), _stream(stream)),
                   "rtlynx_linear_host")
+
+
+def rtlynx_kernel_launches(M, D_in, D_out, R, mode) -> int:
+    return int(lib().rtlynx_kernel_launches(M, D_in, D_out, R, mode))
 
 
 def rtlynx_stream_status(stream=None) -> int:

@@ -188,11 +188,21 @@ static int cached_workspace(int dev, cudaStream_t stream, size_t bytes, void** o
     return RTLYNX_OK;
 }
 
+// Which prologue runs: the one-pass cluster kernel (returns its cluster size)
+// or the two-pass path (returns 0).
+static int prologue_plan(const Dims& d, int num_sms, int* cpc, int* lbs) {
+    // The one-pass cluster prologue re-reads L_B per 64 tokens; it is used
+    // while X is small enough to stay in L2.  Beyond that the two-pass path,
+    // whose second read of X is the cheaper cost, is faster.
+    const bool small_x = static_cast<double>(d.M) * static_cast<double>(d.K) * 2.0 <= 48.0 * (1 << 20);
+    return small_x ? pick_cluster_split(d, num_sms, cpc, lbs) : 0;
+}
+
 static int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
                         int num_sms, cudaStream_t stream) {
-    int cpc = 0;
-    const int cs = pick_cluster_split(d, num_sms, &cpc);
-    if (cs > 0) return launch_sparsify_cluster(d, cs, cpc, X, L_B, ws, err, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;
+    int cpc = 0, lbs = 0;
+    const int cs = prologue_plan(d, num_sms, &cpc, &lbs);
+    if (cs > 0) return launch_sparsify_cluster(d, cs, cpc, lbs, X, L_B, ws, err, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;
     if (launch_norms_lora_down(d, X, L_B, ws, err, stream)) return RTLYNX_ERR_CUDA;
     if (launch_compress(d, X, ws, stream)) return RTLYNX_ERR_CUDA;
     return RTLYNX_OK;
@@ -329,6 +339,17 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
         cudaSuccess)
         return RTLYNX_ERR_CUDA;
     return RTLYNX_OK;
+}
+
+int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode) {
+    if (mode == RTLYNX_MODE_DENSE_SKIP) return (M > 0 && D_in > 0 && D_out > 0) ? 1 : 0;
+    if (mode != RTLYNX_MODE_SPARSE || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8) return 0;
+    DeviceInfo* di = nullptr;
+    const int sms = current_device(&di) == RTLYNX_OK ? di->num_sms : 148;
+    const Dims d = make_dims(M, D_in, D_out, R, sms);
+    int cpc = 0, lbs = 0;
+    if (prologue_plan(d, sms, &cpc, &lbs) > 0) return 2;  // cluster prologue + GEMM
+    return R > 0 ? 4 : 3;                                 // norms (+ T finalize) + compress + GEMM
 }
 
 int rtlynx_stream_status(void* stream_) {

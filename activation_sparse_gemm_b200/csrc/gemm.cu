@@ -343,6 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (lane == 0) bulk_wait_all();
     }
 
+    __syncwarp();  // reconverge the role warps before the cluster barrier
     // After an abort, give copies still in flight time to land before the
     // shared memory they target is released.
     if (error_seen(err)) {

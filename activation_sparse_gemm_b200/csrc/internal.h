@@ -61,8 +61,8 @@ int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const 
 int launch_compress(const Dims& d, const void* X, const Workspace& ws, cudaStream_t stream);
 // One-pass prologue through CTA clusters; pick_cluster_split returns the
 // cluster size (0 when the slice does not fit and the two-pass path is used).
-int pick_cluster_split(const Dims& d, int num_sms, int* chunks_per_cta);
-int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, const void* X, const void* L_B,
+int pick_cluster_split(const Dims& d, int num_sms, int* chunks_per_cta, int* lb_slots);
+int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, int lb_slots, const void* X, const void* L_B,
                             const Workspace& ws, int* err, cudaStream_t stream);
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream);

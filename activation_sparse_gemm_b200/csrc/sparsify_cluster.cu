@@ -26,7 +26,7 @@
 namespace rtlynx {
 
 constexpr int kRB = 64;                   // tokens per cluster
-constexpr int kCThreads = 256;
+constexpr int kCThreads = 576;             // 2 role warps + 16 worker warps
 constexpr int kXTile = kRB * 128;         // one 64 x 64 bf16 tile (128 B rows): 8 KB
 constexpr int kMaxTiles = 64;
 
@@ -34,6 +34,7 @@ struct ClusterArgs {
     int M, K;
     int64_t M_pad, Kc_pad;
     int k_chunks, chunks_per_cta, R_pad;
+    int lb_slots;  // L_B tiles resident at once (the whole slice when it fits)
     uint16_t* vals;
     uint8_t* meta;
     float* s_out;
@@ -41,16 +42,20 @@ struct ClusterArgs {
     int* err;
 };
 
-// Shared-memory bytes the kernel needs for a given split.
-__host__ __device__ inline int cluster_smem_bytes(int chunks_per_cta, int R_pad) {
+// Shared-memory bytes the kernel needs for a given split and L_B ring.
+__host__ __device__ inline int cluster_body_bytes(int chunks_per_cta, int R_pad, int lb_slots) {
     const int x = 2 * chunks_per_cta * kXTile;
-    const int lb = R_pad > 0 ? 2 * R_pad * 128 : 0;
+    const int lb = R_pad > 0 ? lb_slots * R_pad * 128 : 0;
     // the T MMA reads 128 rows from the last 64-row X tile: keep 8 KB after it
     const int tail = (R_pad > 0 && lb < kXTile) ? kXTile - lb : 0;
-    int tpart = kRB * R_pad * 4;
-    int body = x + lb + tail;
-    if (tpart > body) body = tpart;
-    return body + kRB * 16 + kRB * 4 + 1024 /*barriers*/ + 1024 /*align*/;
+    const int tpart = kRB * (R_pad + 1) * 4;
+    const int body = x + lb + tail;
+    return tpart > body ? tpart : body;
+}
+
+__host__ __device__ inline int cluster_smem_bytes(int chunks_per_cta, int R_pad, int lb_slots) {
+    return cluster_body_bytes(chunks_per_cta, R_pad, lb_slots) + kRB * 16 + kRB * 4 + 2048 /*barriers*/ +
+           1024 /*align*/;
 }
 
 template <bool LORA>
@@ -72,19 +77,17 @@ __global__ void __launch_bounds__(kCThreads, 1)
 
     const int x_bytes = 2 * a.chunks_per_cta * kXTile;
     const int lb_slot = LORA ? a.R_pad * 128 : 0;
+    const int LBS = a.lb_slots;
     uint8_t* sX = smem;
     uint8_t* sLB = smem + x_bytes;
-    const int lb_bytes = 2 * lb_slot;
-    const int tail = (LORA && lb_bytes < kXTile) ? kXTile - lb_bytes : 0;
-    int body = x_bytes + lb_bytes + tail;
-    if (kRB * a.R_pad * 4 > body) body = kRB * a.R_pad * 4;
+    const int body = cluster_body_bytes(a.chunks_per_cta, LORA ? a.R_pad : 0, LBS);
     float* sTpart = reinterpret_cast<float*>(smem);  // reuses X / L_B after compression
     double* sPart = reinterpret_cast<double*>(smem + body);          // [kRB][2]
     float* sS = reinterpret_cast<float*>(smem + body + kRB * 16);     // [kRB]
     uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + body + kRB * 16 + kRB * 4);
     uint64_t* full_lb = full_x + kMaxTiles;
-    uint64_t* empty_lb = full_lb + 2;
-    uint64_t* t_done = empty_lb + 2;
+    uint64_t* empty_lb = full_lb + kMaxTiles;
+    uint64_t* t_done = empty_lb + kMaxTiles;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(t_done + 1);
 
     uint32_t tmem_cols = 32;
@@ -92,10 +95,10 @@ __global__ void __launch_bounds__(kCThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < ntiles; ++i) mbar_init(&full_x[i], 1);
-        mbar_init(&full_lb[0], 1);
-        mbar_init(&full_lb[1], 1);
-        mbar_init(&empty_lb[0], 1);
-        mbar_init(&empty_lb[1], 1);
+        for (int i = 0; i < LBS; ++i) {
+            mbar_init(&full_lb[i], 1);
+            mbar_init(&empty_lb[i], 1);
+        }
         mbar_init(t_done, 1);
         fence_mbar_init();
         prefetch_tmap(&tmX);
@@ -119,8 +122,8 @@ __global__ void __launch_bounds__(kCThreads, 1)
         }
         if (LORA) {
             for (int i = 0; i < ntiles; ++i) {
-                const int slot = i & 1;
-                if (!mbar_wait(&empty_lb[slot], ((i >> 1) & 1) ^ 1u, err)) break;
+                const int slot = i % LBS, pass = i / LBS;
+                if (!mbar_wait(&empty_lb[slot], (pass & 1) ^ 1u, err)) break;
                 mbar_arrive_expect_tx(&full_lb[slot], lb_slot);
                 tma_load_2d(sLB + slot * lb_slot, &tmLB, &full_lb[slot], k_begin + i * 64, 0);
             }
@@ -130,9 +133,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
         const uint64_t dX = make_sdesc(smem_u32(sX), 16, 1024, kSw128);
         const uint64_t dL = make_sdesc(smem_u32(sLB), 16, 1024, kSw128);
         for (int i = 0; i < ntiles; ++i) {
-            const int slot = i & 1;
+            const int slot = i % LBS, pass = i / LBS;
             if (!mbar_wait(&full_x[i], 0, err)) break;
-            if (!mbar_wait(&full_lb[slot], (i >> 1) & 1, err)) break;
+            if (!mbar_wait(&full_lb[slot], pass & 1, err)) break;
             tc_fence_after();
             const uint64_t ax = dX + static_cast<uint64_t>((i * kXTile) >> 4);
             const uint64_t bl = dL + static_cast<uint64_t>((slot * lb_slot) >> 4);
@@ -142,41 +145,42 @@ __global__ void __launch_bounds__(kCThreads, 1)
         }
         tc_commit(t_done);
     }
+    __syncwarp();  // reconverge the role warps before any block-wide barrier
 
-    // ---------------------------------------------------------------- partial norms (all threads)
-    {
-        const int r = threadIdx.x >> 2;  // token within the cluster's 64
-        const int q = threadIdx.x & 3;   // quarter of each 64-wide tile row
+    // ---------------------------------------------------------------- partial norms (worker warps 2..17)
+    // worker w handles token r = w / 8 and the 16-byte unit u = w % 8 of each
+    // 128-byte tile row (two groups of four channels per tile)
+    const int wr = (threadIdx.x - 64) >> 3;
+    const int wu = (threadIdx.x - 64) & 7;
+    const uint32_t unit_off = static_cast<uint32_t>(wr * 128 + ((wu ^ (wr & 7)) << 4));
+    if (warp >= 2) {
         double nx = 0.0, nt = 0.0;
         for (int i = 0; i < ntiles; ++i) {
             uint32_t ok = 1;
             if (lane == 0) ok = mbar_wait(&full_x[i], 0, err) ? 1u : 0u;
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
-            const uint8_t* row = sX + i * kXTile + r * 128;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c = 2 * q + h;
-                const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
-                group_energy(v.x, v.y, nx, nt);
-                group_energy(v.z, v.w, nx, nt);
-            }
+            const uint4 v = *reinterpret_cast<const uint4*>(sX + i * kXTile + unit_off);
+            group_energy(v.x, v.y, nx, nt);
+            group_energy(v.z, v.w, nx, nt);
         }
-        // fixed-order combine of the four quarters of the row
-        nx += __shfl_xor_sync(0xFFFFFFFFu, nx, 1);
-        nt += __shfl_xor_sync(0xFFFFFFFFu, nt, 1);
-        nx += __shfl_xor_sync(0xFFFFFFFFu, nx, 2);
-        nt += __shfl_xor_sync(0xFFFFFFFFu, nt, 2);
-        if (q == 0) {
-            sPart[2 * r] = nx;
-            sPart[2 * r + 1] = nt;
+        // fixed-order combine of the eight units of the token (every lane ends with the same sums)
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            nx += __shfl_xor_sync(0xFFFFFFFFu, nx, o);
+            nt += __shfl_xor_sync(0xFFFFFFFFu, nt, o);
+        }
+        if (wu == 0) {
+            sPart[2 * wr] = nx;
+            sPart[2 * wr + 1] = nt;
         }
     }
     cluster_sync();
 
     // ---------------------------------------------------------------- s, summed over the cluster in rank order
-    if (threadIdx.x < kRB) {
-        const uint32_t base = smem_u32(&sPart[2 * threadIdx.x]);
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + kRB) {
+        const int r = threadIdx.x - 64;
+        const uint32_t base = smem_u32(&sPart[2 * r]);
         double nx = 0.0, nt = 0.0;
         for (uint32_t j = 0; j < csize; ++j) {
             const uint32_t addr = mapa_shared(base, j);
@@ -184,38 +188,31 @@ __global__ void __launch_bounds__(kCThreads, 1)
             nt += ld_shared_cluster_f64(addr + 8);
         }
         const float s = static_cast<float>(sqrt(nx) / (sqrt(nt) + 1e-8));
-        sS[threadIdx.x] = s;
-        if (rank == 0) a.s_out[row0 + threadIdx.x] = s;
+        sS[r] = s;
+        if (rank == 0) a.s_out[row0 + r] = s;
     }
     __syncthreads();
 
     // ---------------------------------------------------------------- compress from shared memory
-    {
-        const int pieces = 4 * ntiles;  // 16-wide K pieces per token
-        for (int idx = threadIdx.x; idx < kRB * pieces; idx += kCThreads) {
-            const int r = idx / pieces;
-            const int p = idx - r * pieces;
-            const int tile = p >> 2, pp = p & 3;
-            const uint8_t* row = sX + tile * kXTile + r * 128;
-            const uint4 lo = *reinterpret_cast<const uint4*>(row + (((2 * pp) ^ (r & 7)) << 4));
-            const uint4 hi = *reinterpret_cast<const uint4*>(row + (((2 * pp + 1) ^ (r & 7)) << 4));
-            const float s = sS[r];
-            uint4 out;
-            uint32_t nib = compress_group(lo.x, lo.y, s, out.x);
-            nib |= compress_group(lo.z, lo.w, s, out.y) << 4;
-            nib |= compress_group(hi.x, hi.y, s, out.z) << 8;
-            nib |= compress_group(hi.z, hi.w, s, out.w) << 12;
-            const int64_t grow = row0 + r;
-            const int64_t k = k_begin + p * 16;
-            *reinterpret_cast<uint4*>(a.vals + grow * a.Kc_pad + (k >> 1)) = out;
-            const int m = static_cast<int>(grow & 127);
-            const int m0 = m & 7, m1 = (m >> 3) & 1, m2 = m >> 4;
-            const int kk = static_cast<int>(k & 127);
-            const int k2 = kk >> 5, k1 = (kk >> 4) & 1;
-            const int dp = m0 + 8 * k1 + 16 * m2;
-            uint16_t* w = reinterpret_cast<uint16_t*>(a.meta + ((grow >> 7) * a.k_chunks + (k >> 7)) * kChunkBytes +
-                                                      dp * 16 + k2 * 4 + m1 * 2);
-            *w = static_cast<uint16_t>(nib);
+    if (warp >= 2) {
+        const float s = sS[wr];
+        const int64_t grow = row0 + wr;
+        // metadata: token m of its 128-token block, 8 channels per unit = two nibbles = one byte
+        const int m = static_cast<int>(grow & 127);
+        const int m0 = m & 7, m1 = (m >> 3) & 1, m2 = m >> 4;
+        uint8_t* meta_blk = a.meta + (grow >> 7) * a.k_chunks * kChunkBytes;
+        uint2* vrow = reinterpret_cast<uint2*>(a.vals + grow * a.Kc_pad + (k_begin >> 1));
+        for (int i = 0; i < ntiles; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sX + i * kXTile + unit_off);
+            uint2 out;
+            uint32_t nib = compress_group(v.x, v.y, s, out.x);
+            nib |= compress_group(v.z, v.w, s, out.y) << 4;
+            vrow[i * 8 + wu] = out;  // 4 kept values of channels k_begin + 64 i + 8 wu ...
+            const int k = k_begin + i * 64 + wu * 8;  // first channel of the unit
+            const int kk = k & 127;
+            const int dp = m0 + 8 * ((kk >> 4) & 1) + 16 * m2;
+            meta_blk[(k >> 7) * kChunkBytes + dp * 16 + (kk >> 5) * 4 + m1 * 2 + ((kk >> 3) & 1)] =
+                static_cast<uint8_t>(nib);
         }
     }
 
@@ -241,7 +238,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
                     tmem_ld_wait();
                 }
 #pragma unroll
-                for (int q = 0; q < 32; ++q) sTpart[r * a.R_pad + c + q] = have ? __uint_as_float(v[q]) : 0.0f;
+                for (int q = 0; q < 32; ++q) sTpart[r * (a.R_pad + 1) + c + q] = have ? __uint_as_float(v[q]) : 0.0f;
             }
         }
         tc_fence_before();
@@ -251,7 +248,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
         for (int idx = threadIdx.x; idx < kRB * cols; idx += kCThreads) {
             const int r = idx / cols;
             const int c = c0 + (idx - r * cols);
-            const uint32_t base = smem_u32(&sTpart[r * a.R_pad + c]);
+            const uint32_t base = smem_u32(&sTpart[r * (a.R_pad + 1) + c]);
             float acc = 0.f;
             for (uint32_t j = 0; j < csize; ++j) acc += ld_shared_cluster_f32(mapa_shared(base, j));
             a.T[(row0 + r) * static_cast<int64_t>(a.R_pad) + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
@@ -268,33 +265,46 @@ __global__ void __launch_bounds__(kCThreads, 1)
 // Picks the cluster split: the smallest power-of-two number of CTAs per 64
 // tokens whose slice fits in shared memory and that puts at least two CTAs
 // on every SM.  Returns 0 when no split fits (callers use the two-pass path).
-int pick_cluster_split(const Dims& d, int num_sms, int* chunks_per_cta) {
+int pick_cluster_split(const Dims& d, int num_sms, int* chunks_per_cta, int* lb_slots) {
     const int row_blocks = static_cast<int>(d.M_pad / kRB);
-    auto fits = [&](int cs, int* cpc) {
+    const int R_pad = static_cast<int>(d.R_pad);
+    constexpr int kBudget = 220 * 1024;
+    // Largest L_B ring (up to the whole slice) that fits next to the X slice.
+    auto fit = [&](int cs, int* cpc, int* lbs) {
         *cpc = static_cast<int>((d.k_chunks + cs - 1) / cs);
         if (2 * *cpc > kMaxTiles) return false;
-        if (cluster_smem_bytes(*cpc, static_cast<int>(d.R_pad)) > 225 * 1024) return false;
-        return d.R_pad == 0 || d.R_pad % cs == 0;
+        if (R_pad > 0 && R_pad % cs != 0) return false;
+        if (R_pad == 0) {
+            *lbs = 1;
+            return cluster_smem_bytes(*cpc, 0, 1) <= kBudget;
+        }
+        for (int l = 2 * *cpc; l >= 2; --l) {
+            if (cluster_smem_bytes(*cpc, R_pad, l) <= kBudget) {
+                *lbs = l;
+                return true;
+            }
+        }
+        return false;
     };
-    // portable cluster sizes first; 16 only when nothing smaller fits
-    for (int cs = 1; cs <= 8; cs *= 2) {
-        int cpc = 0;
-        if (!fits(cs, &cpc)) continue;
-        const bool enough = static_cast<int64_t>(cs) * row_blocks >= 2LL * num_sms;
-        if (enough || cs >= d.k_chunks || cs == 8) {
-            *chunks_per_cta = cpc;
-            return cs;
+    int best = 0;
+    for (int pass = 0; pass < 2 && !best; ++pass) {
+        for (int cs = 1; cs <= 16; cs *= 2) {
+            int cpc = 0, lbs = 0;
+            if (!fit(cs, &cpc, &lbs)) continue;
+            if (pass == 0 && R_pad > 0 && lbs < 2 * cpc) continue;  // first try: whole L_B slice resident
+            const bool enough = static_cast<int64_t>(cs) * row_blocks >= 2LL * num_sms;
+            if (enough || cs >= d.k_chunks || cs == 16) {
+                *chunks_per_cta = cpc;
+                *lb_slots = lbs;
+                best = cs;
+                break;
+            }
         }
     }
-    int cpc = 0;
-    if (fits(16, &cpc)) {
-        *chunks_per_cta = cpc;
-        return 16;
-    }
-    return 0;
+    return best;
 }
 
-int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, const void* X, const void* L_B,
+int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, int lb_slots, const void* X, const void* L_B,
                             const Workspace& ws, int* err, cudaStream_t stream) {
     const bool lora = d.R > 0 && L_B != nullptr;
     CUtensorMap tmX, tmLB;
@@ -314,13 +324,14 @@ int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, const voi
     a.Kc_pad = d.Kc_pad;
     a.k_chunks = static_cast<int>(d.k_chunks);
     a.chunks_per_cta = chunks_per_cta;
+    a.lb_slots = lb_slots;
     a.R_pad = lora ? static_cast<int>(d.R_pad) : 0;
     a.vals = ws.vals;
     a.meta = ws.meta;
     a.s_out = ws.s;
     a.T = ws.T;
     a.err = err;
-    const int smem = cluster_smem_bytes(chunks_per_cta, a.R_pad);
+    const int smem = cluster_smem_bytes(chunks_per_cta, a.R_pad, lb_slots);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(d.M_pad / kRB), 1);
     cfg.blockDim = dim3(kCThreads, 1, 1);

@@ -336,10 +336,10 @@ def run_ours(args, wl):
         "e2e": {"value": flop * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "us_per_call": e2e_ms * 1e3},
-        "gpu_launches": kernels_per_step(R) * args.steps,
+        "gpu_launches": rl.rtlynx_kernel_launches(M, K, N, R, rl.MODE_SPARSE) * args.steps,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": sparse_peak, "unit": "TFLOP/s",
                      "frac": achieved / sparse_peak, "traffic": traffic,
-                     "kernel": "rtlynx_gemm_kernel<sparse>",
+                     "kernel": "rtlynx_gemm_pair_kernel<sparse, 240>",
                      "peak_note": f"2 x {peaks_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s): "
                                   "2:4 sparse nominal ratio"},
         "clocks": clocks.summary(),
@@ -354,11 +354,6 @@ def run_ours(args, wl):
         dist.barrier()
         dist.destroy_process_group()
     return 0
-
-
-def kernels_per_step(R):
-    """Our kernels per sparse-mode call: norms/LoRA-down, finalize T (R > 0), compress, GEMM."""
-    return 4 if R > 0 else 3
 
 
 def kernel_rev():

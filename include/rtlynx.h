@@ -117,6 +117,11 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
                        int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* X_dev, void* Y_dev,
                        void* stream);
 
+/* Number of kernels one rtlynx_linear call with these sizes launches (0 for
+ * invalid sizes): the sparse path launches its prologue kernel(s) and the GEMM,
+ * the dense-skip path the GEMM alone. */
+int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode);
+
 /* Synchronizes stream, then returns and clears the current device's error
  * word (RTLYNX_OK or RTLYNX_ERR_DEVICE_TIMEOUT), or RTLYNX_ERR_CUDA. */
 int rtlynx_stream_status(void* stream);
