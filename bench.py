@@ -35,7 +35,7 @@ FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -60,10 +60,10 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
-def oracle_sample(wl, X, W, L_A, L_B, target_s, min_rows=2):
+def oracle_sample(wl, X, W, L_A, L_B, target_s, min_rows=32):
     """Times the CPU oracle on the first n token rows, n chosen for ~target_s of work."""
     import oracle
-    n = min_rows
+    n = min(min_rows, wl.M)
     t0 = time.perf_counter()
     oracle.linear(X, W, L_A, L_B, rows=list(range(n)))
     dt = max(time.perf_counter() - t0, 1e-6)
@@ -314,13 +314,7 @@ def run_ours(args, wl):
     peaks, peaks_kind = load_peaks()
     sparse_peak = 2.0 * peaks["bf16_tflops"]
     achieved = gemm_flop / (gemm_mean / 1e3) / 1e12
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "gemm_sparse_traffic.json")
-    if os.path.exists(prof):
-        with open(prof) as f:
-            tj = json.load(f)
-        if tj.get("workload") == wl.name and tj.get("kernel_rev") == kernel_rev():
-            traffic = tj.get("dram_bytes_per_launch")
+    traffic = profiled_traffic(wl.name)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -354,6 +348,26 @@ def run_ours(args, wl):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per GEMM launch from the committed ncu summary of this
+    workload, or None when there is none or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", f"gemm_sparse_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith(("|", "#", " ")):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("kernel_rev") != kernel_rev():
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def kernel_rev():
