@@ -36,9 +36,11 @@ ERR_DEVICE_TIMEOUT = 5
 ABI_SYMBOLS = (
     "rtlynx_linear", "rtlynx_workspace_size", "rtlynx_linear_ws", "rtlynx_linear_ws_events",
     "rtlynx_workspace_layout",
-    "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_kernel_launches", "rtlynx_stream_status",
-    "rtlynx_status_string", "rtlynx_release",
+    "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_linear_noalloc", "rtlynx_kernel_launches",
+    "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
 )
+
+NOALLOC_MAX_BYTES = 32 << 20
 
 _lib = None
 
@@ -79,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_sparsify_debug.restype = i
         L.rtlynx_linear_host.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i, p, p, p]
         L.rtlynx_linear_host.restype = i
+        L.rtlynx_linear_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i, p, p]
+        L.rtlynx_linear_noalloc.restype = i
         L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
         L.rtlynx_kernel_launches.restype = i
         L.rtlynx_stream_status.argtypes = [p]
@@ -159,6 +163,17 @@ def rtlynx_linear_host(X_host, W, L_A, L_B, Y_host, M, D_in, D_out, R, mode, X_d
     return _check(lib().rtlynx_linear_host(_ptr(X_host), _ptr(W), _ptr(L_A), _ptr(L_B), _ptr(Y_host), M, D_in,
                                            D_out, R, mode, _ptr(X_dev), _ptr(Y_dev), _stream(stream)),
                   "rtlynx_linear_host")
+
+
+def rtlynx_linear_noalloc(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, dev_status=None, stream=None) -> int:
+    """rtlynx_linear without any device allocation: for callers that cannot call
+    cudaMalloc (their memory belongs to another pool, or the call sits on a path
+    that must not synchronize).  The workspace is a static device array of
+    NOALLOC_MAX_BYTES shared by all calls on a device; calls that overlap on the
+    GPU race on it.  dev_status: optional device int32 that receives the
+    device-side timeout code."""
+    return _check(lib().rtlynx_linear_noalloc(_ptr(X), _ptr(W), _ptr(L_A), _ptr(L_B), _ptr(Y), M, D_in, D_out, R,
+                                              mode, _ptr(dev_status), _stream(stream)), "rtlynx_linear_noalloc")
 
 
 def rtlynx_kernel_launches(M, D_in, D_out, R, mode) -> int:

@@ -98,6 +98,19 @@ int validate(const void* X, const void* W, const void* L_A, const void* L_B, con
 
 }  // namespace
 
+bool ensure_tmap_encoder() {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return false;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    return true;
+}
+
 int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                    CUtensorMapSwizzle swizzle) {
@@ -155,7 +168,7 @@ WsLayout make_ws_layout(const Dims& d) {
     return l;
 }
 
-static Workspace carve(void* base, const WsLayout& l) {
+Workspace carve(void* base, const WsLayout& l) {
     uint8_t* b = static_cast<uint8_t*>(base);
     Workspace w;
     w.vals = reinterpret_cast<uint16_t*>(b + l.vals);
@@ -190,7 +203,7 @@ static int cached_workspace(int dev, cudaStream_t stream, size_t bytes, void** o
 
 // Which prologue runs: the one-pass cluster kernel (returns its cluster size)
 // or the two-pass path (returns 0).
-static int prologue_plan(const Dims& d, int num_sms, int* cpc, int* lbs) {
+int prologue_plan(const Dims& d, int num_sms, int* cpc, int* lbs) {
     // The one-pass cluster prologue re-reads L_B per 64 tokens; it is used
     // while X is small enough to stay in L2.  Beyond that the two-pass path,
     // whose second read of X is the cheaper cost, is faster.
@@ -198,8 +211,8 @@ static int prologue_plan(const Dims& d, int num_sms, int* cpc, int* lbs) {
     return small_x ? pick_cluster_split(d, num_sms, cpc, lbs) : 0;
 }
 
-static int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
-                        int num_sms, cudaStream_t stream) {
+int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
+                 cudaStream_t stream) {
     int cpc = 0, lbs = 0;
     const int cs = prologue_plan(d, num_sms, &cpc, &lbs);
     if (cs > 0) return launch_sparsify_cluster(d, cs, cpc, lbs, X, L_B, ws, err, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;

@@ -66,6 +66,13 @@ int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, int lb_sl
                             const Workspace& ws, int* err, cudaStream_t stream);
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream);
+// Shared by the entry points (api.cu).
+bool ensure_tmap_encoder();
+Workspace carve(void* base, const WsLayout& l);
+int prologue_plan(const Dims& d, int num_sms, int* chunks_per_cta, int* lb_slots);
+int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
+                 cudaStream_t stream);
+
 int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,
                         cudaStream_t stream);
 

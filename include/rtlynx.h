@@ -117,6 +117,37 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
                        int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* X_dev, void* Y_dev,
                        void* stream);
 
+/* Largest workspace rtlynx_linear_noalloc can use (32 MiB). */
+#define RTLYNX_NOALLOC_MAX_BYTES (32u << 20)
+
+/*
+ * rtlynx_linear_noalloc - rtlynx_linear for callers that cannot allocate
+ * device memory.  (The RT-Lynx pages have no counterpart: this is a
+ * deployment entry point.)
+ *
+ * Some callers cannot call cudaMalloc where they run the layer: a serving
+ * engine that has handed all device memory to its own pool, code whose
+ * allocations must go through an allocator this library does not see, or a
+ * latency-critical path where cudaMalloc, which may synchronize the device,
+ * is not acceptable.  This entry point allocates nothing.  Its workspace is a
+ * static device array of RTLYNX_NOALLOC_MAX_BYTES that every GPU using this
+ * entry point holds until the process exits; problems whose workspace
+ * (rtlynx_workspace_size) is larger are rejected with RTLYNX_ERR_UNSUPPORTED
+ * before anything is launched.
+ *   dev_status  a caller-owned, 4-byte-aligned device int (or NULL): a
+ *               bounded device-side wait that runs out stores
+ *               RTLYNX_ERR_DEVICE_TIMEOUT's device code (1) there; the caller
+ *               zeroes it beforehand and reads it after synchronizing.
+ * Other arguments as rtlynx_linear.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and reads device properties;
+ * make it outside any stream capture.  Every call shares the one array and
+ * rewrites every part it reads, so nothing needs clearing between calls, but
+ * calls that overlap on the GPU (other streams or host threads on the same
+ * device) race on it and must be serialized by the caller.
+ */
+int rtlynx_linear_noalloc(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
+                          int64_t D_in, int64_t D_out, int64_t R, int mode, int* dev_status, void* stream);
+
 /* Number of kernels one rtlynx_linear call with these sizes launches (0 for
  * invalid sizes): the sparse path launches its prologue kernel(s) and the GEMM,
  * the dense-skip path the GEMM alone. */
