@@ -186,20 +186,14 @@ def run_reference(args, wl):
 def run_ours(args, wl):
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     import activation_sparse_gemm_b200 as rl
     from activation_sparse_gemm_b200.inputs import make_inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
+    from activation_sparse_gemm_b200 import dist as rdist
+    world, rank, local = rdist.env_ranks()
+    torch.cuda.set_device(local if world > 1 else 0)
+    rdist.init("nccl", timeout_s=120)
     device = torch.device("cuda", torch.cuda.current_device())
     rl.lib()
 
@@ -216,9 +210,7 @@ def run_ours(args, wl):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = rdist.barrier
 
     def ev():
         e = torch.cuda.Event(enable_timing=True)
@@ -255,11 +247,7 @@ def run_ours(args, wl):
     step_ms = [a.elapsed_time(c) for a, b, c in evs]
     pro_ms = [a.elapsed_time(b) for a, b, c in evs]
     gemm_ms = [b.elapsed_time(c) for a, b, c in evs]
-    ms = statistics.mean(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = rdist.max_over_ranks(statistics.mean(step_ms), device)
 
     # same-run comparisons (not part of the headline value)
     for _ in range(3):
@@ -302,10 +290,7 @@ def run_ours(args, wl):
     status = rl.rtlynx_stream_status(stream)
     if status != rl.OK:
         raise RuntimeError(f"device-side error: {rl.rtlynx_status_string(status)}")
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = rdist.max_over_ranks(e2e_ms, device)
 
     flop = wl.dense_equiv_flop
     value = flop * world / (ms / 1e3) / 1e12
@@ -344,9 +329,7 @@ def run_ours(args, wl):
         line["cpu_baseline"] = oracle_sample(wl, X, W, L_A, L_B, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    rdist.shutdown()
     return 0
 
 
