@@ -37,7 +37,7 @@ ABI_SYMBOLS = (
     "rtlynx_linear", "rtlynx_workspace_size", "rtlynx_linear_ws", "rtlynx_linear_ws_events",
     "rtlynx_workspace_layout",
     "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_linear_noalloc", "rtlynx_kernel_launches",
-    "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
+    "rtlynx_wait_selftest", "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
 )
 
 NOALLOC_MAX_BYTES = 32 << 20
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_linear_noalloc.restype = i
         L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
         L.rtlynx_kernel_launches.restype = i
+        L.rtlynx_wait_selftest.argtypes = [i64, p]
+        L.rtlynx_wait_selftest.restype = i
         L.rtlynx_stream_status.argtypes = [p]
         L.rtlynx_stream_status.restype = i
         L.rtlynx_status_string.argtypes = [i]
@@ -178,6 +180,10 @@ def rtlynx_linear_noalloc(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, dev_status
 
 def rtlynx_kernel_launches(M, D_in, D_out, R, mode) -> int:
     return int(lib().rtlynx_kernel_launches(M, D_in, D_out, R, mode))
+
+
+def rtlynx_wait_selftest(limit_ns, stream=None) -> int:
+    return _check(lib().rtlynx_wait_selftest(int(limit_ns), _stream(stream)), "rtlynx_wait_selftest")
 
 
 def rtlynx_stream_status(stream=None) -> int:

@@ -365,6 +365,16 @@ int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, in
     return R > 0 ? 4 : 3;                                 // norms (+ T finalize) + compress + GEMM
 }
 
+int rtlynx_wait_selftest(int64_t limit_ns, void* stream_) {
+    if (limit_ns <= 0 || limit_ns > 1000000000) return RTLYNX_ERR_INVALID_ARG;
+    DeviceInfo* di = nullptr;
+    int rc = current_device(&di);
+    if (rc) return rc;
+    return launch_wait_selftest(di->err_word, static_cast<uint64_t>(limit_ns), static_cast<cudaStream_t>(stream_))
+               ? RTLYNX_ERR_CUDA
+               : RTLYNX_OK;
+}
+
 int rtlynx_stream_status(void* stream_) {
     DeviceInfo* di = nullptr;
     int rc = current_device(&di);

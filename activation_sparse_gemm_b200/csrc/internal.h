@@ -73,6 +73,7 @@ int prologue_plan(const Dims& d, int num_sms, int* chunks_per_cta, int* lb_slots
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
                  cudaStream_t stream);
 
+int launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t stream);
 int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,
                         cudaStream_t stream);
 

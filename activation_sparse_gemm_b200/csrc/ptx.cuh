@@ -81,18 +81,25 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 
 constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms per suspended try
 
-// Wait until the phase with the given parity has completed.  Bounded.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// Wait until the phase with the given parity has completed, at most
+// limit_ns of global time.  Returns false (and records the timeout) when the
+// limit runs out, or when another thread has recorded an error already.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* err, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    const uint32_t hint = limit_ns < kSuspendHintNs ? static_cast<uint32_t>(limit_ns / 4 + 1) : kSuspendHintNs;
     while (true) {
-        if (mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
+        if (mbar_try_wait_hint(bar, parity, hint)) return true;
         if (error_seen(err)) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             record_error(err, RTLYNX_DEV_TIMEOUT);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+    return mbar_wait_limit(bar, parity, err, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA / bulk copies

@@ -153,6 +153,12 @@ int rtlynx_linear_noalloc(const void* X, const void* W, const void* L_A, const v
  * the dense-skip path the GEMM alone. */
 int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode);
 
+/* Self-test of the device-side failure detection: launches one thread that
+ * waits on a barrier nothing arrives on.  The wait gives up after limit_ns
+ * (1 .. 1e9), records RTLYNX_ERR_DEVICE_TIMEOUT in the device error word and
+ * returns; the next rtlynx_stream_status() on the stream reports it. */
+int rtlynx_wait_selftest(int64_t limit_ns, void* stream);
+
 /* Synchronizes stream, then returns and clears the current device's error
  * word (RTLYNX_OK or RTLYNX_ERR_DEVICE_TIMEOUT), or RTLYNX_ERR_CUDA. */
 int rtlynx_stream_status(void* stream);

@@ -82,3 +82,8 @@ def test_python_binding_raises_on_error(lib):
 def test_workspace_size_zero_for_dense_and_invalid(lib):
     assert rl.rtlynx_workspace_size(128, 256, 256, 64, rl.MODE_DENSE_SKIP) == 0
     assert rl.rtlynx_workspace_size(128, 250, 256, 64, rl.MODE_SPARSE) == 0
+
+
+def test_wait_selftest_rejects_bad_limits_without_launch(lib):
+    for limit in (0, -1, 2_000_000_000):
+        assert lib.rtlynx_wait_selftest(limit, None) == rl.ERR_INVALID_ARG

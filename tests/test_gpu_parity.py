@@ -237,3 +237,17 @@ def test_full_workload_sampled(name):
     if name == "mlp_down":
         Yd = run_linear(X, W, None, None, mode=rl.MODE_DENSE_SKIP)
         assert_y_close(Yd[rows], oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP, rows=rows), "mlp_down dense")
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A device wait on a barrier nobody arrives on gives up, reports
+    DEVICE_TIMEOUT through the status word, and the context keeps working."""
+    import torch
+    rl.rtlynx_wait_selftest(5_000_000)  # 5 ms
+    assert rl.rtlynx_stream_status() == rl.ERR_DEVICE_TIMEOUT
+    assert rl.rtlynx_stream_status() == rl.OK  # the status word was cleared
+    X, W, L_A, L_B = make_custom(130, 256, 128, 32, seed=77)
+    Y = run_linear(X, W, L_A, L_B)
+    assert_y_close(Y, oracle.linear(X, W, L_A, L_B), "after timeout", edge=True)
+    torch.cuda.synchronize()
