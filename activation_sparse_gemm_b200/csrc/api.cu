@@ -138,14 +138,15 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
     d.k_chunks = (K + kChunkK - 1) / kChunkK;
     d.Kc_pad = d.k_chunks * (kChunkK / 2);
     d.R_pad = R > 0 ? (R + 63) / 64 * 64 : 0;
-    // Enough CTAs in the norm / LoRA-down pass to cover the GPU about twice,
-    // every split holding at least one K tile.
-    int64_t target = 2 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148);
-    int64_t ns = (target + d.m_blocks - 1) / d.m_blocks;
-    if (ns < 1) ns = 1;
-    if (ns > d.k_tiles) ns = d.k_tiles;
-    const int64_t tps = (d.k_tiles + ns - 1) / ns;
-    d.nsplit = (d.k_tiles + tps - 1) / tps;
+    // Streaming prologue: one CTA per SM over the row-block x K-tile grid.
+    d.kt2 = 2 * d.k_chunks;
+    const int64_t total = d.m_blocks * d.kt2;
+    const int64_t sms = num_sms > 0 ? num_sms : 148;
+    d.grid1 = total < sms ? total : sms;
+    // A row block's kt2 tiles meet at most (kt2 - 2) / L + 2 runs when every
+    // run holds at least L = floor(total / grid1) tiles.
+    const int64_t run = total / d.grid1;
+    d.max_segs = (d.kt2 - 2) / run + 2;
     return d;
 }
 
@@ -161,9 +162,9 @@ WsLayout make_ws_layout(const Dims& d) {
     l.T = off;
     off = align256(off + static_cast<size_t>(d.M_pad) * d.R_pad * 2);
     l.part_norm = off;
-    off = align256(off + static_cast<size_t>(d.nsplit) * d.M_pad * 2 * 8);
+    off = align256(off + static_cast<size_t>(d.max_segs) * d.M_pad * 2 * 8);
     l.part_T = off;
-    off = align256(off + static_cast<size_t>(d.nsplit) * d.M_pad * d.R_pad * 4);
+    off = align256(off + static_cast<size_t>(d.max_segs) * d.M_pad * d.R_pad * 4);
     l.total = off;
     return l;
 }
@@ -203,22 +204,10 @@ static int cached_workspace(int dev, cudaStream_t stream, size_t bytes, void** o
 
 // Which prologue runs: the one-pass cluster kernel (returns its cluster size)
 // or the two-pass path (returns 0).
-int prologue_plan(const Dims& d, int num_sms, int* cpc, int* lbs) {
-    // The one-pass cluster prologue re-reads L_B per 64 tokens; it is used
-    // while X is small enough to stay in L2.  Beyond that the two-pass path,
-    // whose second read of X is the cheaper cost, is faster.
-    const bool small_x = static_cast<double>(d.M) * static_cast<double>(d.K) * 2.0 <= 48.0 * (1 << 20);
-    return small_x ? pick_cluster_split(d, num_sms, cpc, lbs) : 0;
-}
-
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
                  cudaStream_t stream) {
-    int cpc = 0, lbs = 0;
-    const int cs = prologue_plan(d, num_sms, &cpc, &lbs);
-    if (cs > 0) return launch_sparsify_cluster(d, cs, cpc, lbs, X, L_B, ws, err, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;
-    if (launch_norms_lora_down(d, X, L_B, ws, err, stream)) return RTLYNX_ERR_CUDA;
-    if (launch_compress(d, X, ws, stream)) return RTLYNX_ERR_CUDA;
-    return RTLYNX_OK;
+    (void)num_sms;  // the split is fixed in make_dims
+    return launch_sparsify(d, X, L_B, ws, err, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;
 }
 
 }  // namespace rtlynx
@@ -357,12 +346,7 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
 int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode) {
     if (mode == RTLYNX_MODE_DENSE_SKIP) return (M > 0 && D_in > 0 && D_out > 0) ? 1 : 0;
     if (mode != RTLYNX_MODE_SPARSE || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8) return 0;
-    DeviceInfo* di = nullptr;
-    const int sms = current_device(&di) == RTLYNX_OK ? di->num_sms : 148;
-    const Dims d = make_dims(M, D_in, D_out, R, sms);
-    int cpc = 0, lbs = 0;
-    if (prologue_plan(d, sms, &cpc, &lbs) > 0) return 2;  // cluster prologue + GEMM
-    return R > 0 ? 4 : 3;                                 // norms (+ T finalize) + compress + GEMM
+    return 3;  // streaming sparsify pass, per-token scale pass, GEMM
 }
 
 int rtlynx_wait_selftest(int64_t limit_ns, void* stream_) {

@@ -24,8 +24,18 @@ struct Dims {
     int64_t k_chunks;     // ceil(K / kChunkK)
     int64_t Kc_pad;       // compressed row length in elements = k_chunks * kChunkK / 2
     int64_t R_pad;        // R rounded up to 64 (0 when R == 0)
-    int64_t nsplit;       // K-splits of the norm / LoRA-down pass
+    int64_t kt2;          // 64-wide K tiles per row block in the prologue = 2 * k_chunks
+    int64_t grid1;        // CTAs of the streaming prologue pass
+    int64_t max_segs;     // most CTAs whose tile runs meet one row block (partial-sum slots)
 };
+
+// The streaming prologue cuts the m_blocks * kt2 tiles into `grid` contiguous
+// runs: CTA c takes tiles [stream_begin(c), stream_begin(c + 1)), and tile t
+// belongs to CTA stream_owner(t).
+__host__ __device__ inline int64_t stream_begin(int64_t c, int64_t total, int64_t grid) { return c * total / grid; }
+__host__ __device__ inline int64_t stream_owner(int64_t t, int64_t total, int64_t grid) {
+    return ((t + 1) * grid - 1) / total;
+}
 
 // Byte offsets of the sparse-mode workspace regions (each 256-byte aligned).
 struct WsLayout {
@@ -40,8 +50,8 @@ struct Workspace {
     uint8_t* meta;        // [m_blocks, k_chunks, 2048] metadata chunks in tensor-memory order
     float* s;             // [M_pad] per-token scale
     uint16_t* T;          // [M_pad, R_pad] bf16, X L_B^T
-    double* part_norm;    // [nsplit, M_pad, 2] partial sum of x^2 and of kept x^2
-    float* part_T;        // [nsplit, M_pad, R_pad] partial X L_B^T
+    double* part_norm;    // [max_segs, M_pad, 2] partial sums of x^2 and of kept x^2
+    float* part_T;        // [max_segs, M_pad, R_pad] partial X L_B^T
 };
 
 // Tensor-map encoding through the driver entry point (no libcuda link needed).
@@ -56,20 +66,14 @@ inline int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inne
 }
 
 // Launchers; each returns a cudaError_t value (0 on success).
-int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
-                           cudaStream_t stream);
-int launch_compress(const Dims& d, const void* X, const Workspace& ws, cudaStream_t stream);
-// One-pass prologue through CTA clusters; pick_cluster_split returns the
-// cluster size (0 when the slice does not fit and the two-pass path is used).
-int pick_cluster_split(const Dims& d, int num_sms, int* chunks_per_cta, int* lb_slots);
-int launch_sparsify_cluster(const Dims& d, int cs, int chunks_per_cta, int lb_slots, const void* X, const void* L_B,
-                            const Workspace& ws, int* err, cudaStream_t stream);
+// The sparsify prologue: two launches (streaming pass, then per-token scale).
+int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
+                    cudaStream_t stream);
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream);
 // Shared by the entry points (api.cu).
 bool ensure_tmap_encoder();
 Workspace carve(void* base, const WsLayout& l);
-int prologue_plan(const Dims& d, int num_sms, int* chunks_per_cta, int* lb_slots);
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
                  cudaStream_t stream);
 

@@ -3,21 +3,26 @@
 // step 4 items (1)-(3): mask decision, Top-K, compression to the sparse tensor
 // core layout), plus the LoRA down-projection T = X L_B^T of step 2.
 //
-// Pass 1  norms_lora_down   grid (row block of 128 tokens, K-split).
-//         TMA streams 128 x 64 tiles of X (128B swizzle) and 64-wide tiles of
-//         L_B.  Four warps read each X tile from shared memory, one token per
-//         thread, and accumulate sum(x^2) and sum(x~^2) in double from exact
-//         squares (the kept entries are the two largest magnitudes of each
-//         group; ties do not change the sum).
-//         From the SAME shared-memory tile one thread issues dense tcgen05.mma
-//         (M = 128, N = R) for the partial T.  Partial sums go to the workspace.
-// Pass 2  compress          grid (16-token slab, 256-wide K block).
-//         Sums the partial norms in a fixed order, s = ||x|| / (||x~|| + 1e-8),
-//         applies the exact 2-of-4 rule (integer magnitude compares, ties to the
-//         lower index), rounds s*x once to bf16, and writes the kept values
-//         row-major and the metadata in the order tcgen05.cp copies it into
-//         tensor memory.
-// Pass 3  finalize_T        sums the partial T in a fixed order and rounds to bf16.
+// Pass 1  sparsify_stream   persistent, one CTA per SM.
+//         The (row block of 128 tokens) x (64-wide K tile) grid of X is cut
+//         into equal contiguous runs, one per CTA.  A TMA producer streams the
+//         CTA's tiles (and the matching 64-wide tiles of L_B) through a ring of
+//         shared-memory stages.  Sixteen math warps rank every group of four
+//         once: the 2-of-4 rule (integer magnitude compares, ties to the lower
+//         index) gives the metadata nibble and the two kept entries, which are
+//         written unscaled; the same ranking gives the exact squares for
+//         sum(x^2) and sum(x~^2), accumulated in double (a tile holding zero
+//         or subnormal entries takes a converting path, chosen per warp).  One thread issues
+//         dense tcgen05.mma (M = 128, N = R) from the same shared-memory tiles
+//         into one of two tensor-memory accumulators.  Where a run crosses a
+//         row block, the partial norms and the partial T of the finished
+//         segment go to the workspace.
+// Pass 2  scale             one warp per token.
+//         Sums the token's partial norms in segment order,
+//         s = ||x|| / (||x~|| + 1e-8) in float, rescales the kept entries in
+//         place (s*x rounded once to bf16, nearest even), and sums the partial
+//         T in segment order, rounded to bf16.
+// Every reduction runs in a fixed order, so results are deterministic.
 //
 // Metadata chunk (128 tokens x 128 logical K, 2048 bytes), for token m in the
 // row block (m0 = m % 8, m1 = (m / 8) % 2, m2 = m / 16) and logical k in the
@@ -31,55 +36,74 @@
 
 namespace rtlynx {
 
-// ---------------------------------------------------------------- pass 1
-struct NormArgs {
-    int M;
-    int64_t M_pad;
-    int k_tiles, tiles_per_split, R_pad;
+constexpr int kStreamThreads = 576;  // warp 0 TMA, warp 1 MMA, warps 2-17 math
+constexpr int kMathWarps = 16;
+constexpr int kXTileBytes = kBM * kBK * 2;  // 16 KB
+
+struct StreamArgs {
+    int64_t M_pad, Kc_pad, total_tiles, grid;
+    int kt2, k_chunks, R_pad, stages;
+    uint16_t* vals;
+    uint8_t* meta;
     double* part_norm;
     float* part_T;
     int* err;
 };
 
-constexpr int kNormStages = 4;
-constexpr int kNormThreads = 192;
-constexpr int kXTileBytes = kBM * kBK * 2;  // 16 KB
+// Bytes of one ring stage: a 128 x 64 tile of X and, with LoRA, a R_pad x 64
+// tile of L_B (both multiples of 1024, as the 128-byte swizzle wants).
+__host__ __device__ inline int stream_stage_bytes(int R_pad) { return kXTileBytes + R_pad * kBK * 2; }
 
-__host__ __device__ inline int norm_stage_bytes(int R_pad) {
-    return ((kXTileBytes + R_pad * kBK * 2 + 1023) / 1024) * 1024;
+// Every lane of the warp waits; the warp goes on only if all of them saw the
+// phase complete.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* err) {
+    const bool ok = mbar_wait(bar, parity, err);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// stream_owner with a 32-bit division whenever the operands fit.
+__device__ __forceinline__ int64_t stream_owner_dev(int64_t t, int64_t total, int64_t grid) {
+    const uint64_t num = static_cast<uint64_t>(t + 1) * static_cast<uint64_t>(grid) - 1u;
+    if (num < (1ull << 32) && static_cast<uint64_t>(total) < (1ull << 32))
+        return static_cast<uint32_t>(num) / static_cast<uint32_t>(total);
+    return static_cast<int64_t>(num / static_cast<uint64_t>(total));
 }
 
 template <bool LORA>
-__global__ void __launch_bounds__(kNormThreads, 1)
-    rtlynx_norms_lora_down_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmLB,
-                                  const NormArgs a) {
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    rtlynx_sparsify_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmLB,
+                                  const StreamArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int stage_bytes = norm_stage_bytes(LORA ? a.R_pad : 0);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kNormStages * stage_bytes);
-    uint64_t* empty = full + kNormStages;
-    uint64_t* done_bar = empty + kNormStages;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done_bar + 1);
-    int* consumed_holder = reinterpret_cast<int*>(tmem_holder + 1);
+    const int S = a.stages;
+    const int stage_bytes = stream_stage_bytes(LORA ? a.R_pad : 0);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);
+    uint64_t* empty = full + S;
+    uint64_t* tfull = empty + S;  // [2] accumulator ready for draining
+    uint64_t* tempty = tfull + 2; // [2] accumulator drained
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     int* err = a.err;
-    const int mb = blockIdx.x;
-    const int split = blockIdx.y;
-    const int kt0 = split * a.tiles_per_split;
-    const int kt1 = min(kt0 + a.tiles_per_split, a.k_tiles);
-    const int ntiles = kt1 - kt0;
+    const int64_t cta = blockIdx.x;
+    const int64_t t0 = stream_begin(cta, a.total_tiles, a.grid);
+    const int64_t t1 = stream_begin(cta + 1, a.total_tiles, a.grid);
+    const int64_t kt2 = a.kt2;
     uint32_t tmem_cols = 32;
-    while (tmem_cols < static_cast<uint32_t>(a.R_pad)) tmem_cols <<= 1;
+    while (tmem_cols < static_cast<uint32_t>(2 * a.R_pad)) tmem_cols <<= 1;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNormStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], LORA ? 5 : 4);
+            mbar_init(&empty[s], kMathWarps + (LORA ? 1 : 0));
         }
-        mbar_init(done_bar, 1);
-        *consumed_holder = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(mma_done, 1);
         fence_mbar_init();
         prefetch_tmap(&tmX);
         if (LORA) prefetch_tmap(&tmLB);
@@ -92,109 +116,212 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = LORA ? *tmem_holder : 0u;
-    int issued = 0;
 
+    // Role warps run their loops with all 32 lanes (waits by every lane, the
+    // single-thread actions predicated on lane 0), so every warp reaches the
+    // block-wide barriers converged.  Tile t is row block mb = t / kt2, K tile
+    // kt = t % kt2; the loops step (mb, kt) without dividing.
+    const int64_t mb0 = t0 / kt2;
+    const int kt0 = static_cast<int>(t0 - mb0 * kt2);
     if (warp == 0) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            const uint32_t bytes = kXTileBytes + (LORA ? a.R_pad * kBK * 2 : 0);
-            for (int i = 0; i < ntiles; ++i) {
-                if (!mbar_wait(&empty[stage], phase ^ 1u, err)) break;
-                uint8_t* sX = smem + stage * stage_bytes;
-                mbar_arrive_expect_tx(&full[stage], bytes);
-                tma_load_2d(sX, &tmX, &full[stage], (kt0 + i) * kBK, mb * kBM);
-                if (LORA) tma_load_2d(sX + kXTileBytes, &tmLB, &full[stage], (kt0 + i) * kBK, 0);
-                ++issued;
-                if (++stage == kNormStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-    } else if (warp == 1) {
-        if (LORA && lane == 0) {
-            const uint32_t idesc = make_idesc_bf16(kBM, a.R_pad, false);
-            int stage = 0;
-            uint32_t phase = 0;
-            int consumed = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                if (!mbar_wait(&full[stage], phase, err)) break;
-                tc_fence_after();
-                const uint32_t sX = smem_u32(smem + stage * stage_bytes);
-                const uint32_t sL = sX + kXTileBytes;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint64_t ad = make_sdesc(sX + j * 32, 16, 1024, kSw128);
-                    const uint64_t bd = make_sdesc(sL + j * 32, 16, 1024, kSw128);
-                    mma_f16(tmem_base, ad, bd, idesc, (i | j) != 0);
-                }
-                tc_commit(&empty[stage]);
-                ++consumed;
-                if (++stage == kNormStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            tc_commit(done_bar);
-            mbar_wait(done_bar, 0, nullptr);
-            *consumed_holder = consumed;
-        }
-    } else {
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;  // token row within the block
-        double nx = 0.0, nt = 0.0;
-        int stage = 0;
+        // ------------------------------------------------------------ TMA producer
+        int stage = 0, issued = 0;
         uint32_t phase = 0;
-        int consumed = 0;
-        for (int i = 0; i < ntiles; ++i) {
-            if (!mbar_wait(&full[stage], phase, err)) break;
-            const uint8_t* row = smem + stage * stage_bytes + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
-                group_energy(v.x, v.y, nx, nt);
-                group_energy(v.z, v.w, nx, nt);
+        int64_t mb = mb0;
+        int kt = kt0;
+        for (int64_t t = t0; t < t1; ++t) {
+            if (!warp_wait(&empty[stage], phase ^ 1u, err)) break;
+            if (lane == 0) {
+                uint8_t* sX = smem + stage * stage_bytes;
+                mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(stage_bytes));
+                tma_load_2d(sX, &tmX, &full[stage], kt * kBK, static_cast<int>(mb * kBM));
+                if (LORA) tma_load_2d(sX + kXTileBytes, &tmLB, &full[stage], kt * kBK, 0);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-            ++consumed;
-            if (++stage == kNormStages) {
+            ++issued;
+            if (++stage == S) {
                 stage = 0;
                 phase ^= 1u;
             }
+            if (++kt == a.kt2) {
+                kt = 0;
+                ++mb;
+            }
         }
-        if (!LORA && warp == 2 && lane == 0) *consumed_holder = consumed;
-        const int64_t grow = static_cast<int64_t>(mb) * kBM + r;
-        double* pn = a.part_norm + (static_cast<int64_t>(split) * a.M_pad + grow) * 2;
-        pn[0] = nx;
-        pn[1] = nt;
+        // every issued copy has landed before the CTA may exit
+        for (int q = issued > S ? issued - S : 0; q < issued; ++q)
+            mbar_wait(&full[q % S], static_cast<uint32_t>((q / S) & 1), nullptr);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ LoRA-down MMA issuer
         if (LORA) {
-            if (mbar_wait(done_bar, 0, err)) {
+            const uint32_t idesc = make_idesc_bf16(kBM, a.R_pad, false);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t n = 0;  // segments so far: accumulator n & 1, its use (n >> 1)
+            bool ok = true;
+            int64_t t = t0;
+            int64_t seg_end = min(t1, (mb0 + 1) * kt2);
+            while (ok && t < t1) {
+                const uint32_t b = n & 1u;
+                if (!warp_wait(&tempty[b], ((n >> 1) & 1u) ^ 1u, err)) break;
                 tc_fence_after();
-                float* pt = a.part_T + (static_cast<int64_t>(split) * a.M_pad + grow) * a.R_pad;
-                const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-                for (int c = 0; c < a.R_pad; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(c), v);
-                    tmem_ld_wait();
+                const uint32_t acc = tmem_base + static_cast<uint32_t>(b * a.R_pad);
+                for (bool first = true; t < seg_end; ++t, first = false) {
+                    if (!warp_wait(&full[stage], phase, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t sX = smem_u32(smem + stage * stage_bytes);
+                        const uint32_t sL = sX + kXTileBytes;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 f4 = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-                        *reinterpret_cast<float4*>(pt + c + 4 * q) = f4;
+                        for (int j = 0; j < 4; ++j)
+                            mma_f16(acc, make_sdesc(sX + j * 32, 16, 1024, kSw128),
+                                    make_sdesc(sL + j * 32, 16, 1024, kSw128), idesc, !(first && j == 0));
+                        tc_commit(&empty[stage]);
+                    }
+                    __syncwarp();
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
-                tc_fence_before();
+                if (!ok) break;
+                if (lane == 0) tc_commit(&tfull[b]);
+                __syncwarp();
+                ++n;
+                seg_end = min(t1, seg_end + kt2);
             }
+            if (lane == 0) tc_commit(mma_done);
+            __syncwarp();
+            mbar_wait(mma_done, 0, nullptr);
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------------------------------------ math warps
+        // Thread (row pair, 16-byte unit): rows rA = m0 + 16*m2 and rB = rA + 8
+        // of the block, channels 8u .. 8u+7 of each 64-wide tile.  The eight
+        // lanes of a quarter warp read the eight units of one row (no bank
+        // conflict), and rows rA, rB fill the two halves of the same metadata
+        // word.
+        const int wi = threadIdx.x - 64;
+        const int u = wi & 7, rp = wi >> 3;
+        const int m0 = rp & 7, m2 = rp >> 3;
+        const int rA = m0 + 16 * m2;
+        const uint32_t offA = static_cast<uint32_t>(rA * 128 + ((u ^ m0) << 4));
+        const uint32_t offB = offA + 8 * 128;
+        const int dp = m0 + 8 * ((u >> 1) & 1) + 16 * m2;
+        const bool even = (u & 1) == 0;
+        const bool drain = LORA && warp >= 4 && warp < 8;  // warps reaching tensor-memory lanes 0-127
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t n = 0;  // segments so far (accumulator n & 1)
+        int64_t t = t0;
+        for (int64_t mb = mb0; t < t1; ++mb) {
+            const int64_t seg_end = min(t1, (mb + 1) * kt2);
+            const int64_t seg = cta - stream_owner_dev(mb * kt2, a.total_tiles, a.grid);
+            const int64_t growA = mb * kBM + rA;
+            uint16_t* vA = a.vals + growA * a.Kc_pad + u * 4;
+            uint16_t* vB = vA + 8 * a.Kc_pad;
+            uint8_t* mrow = a.meta + mb * a.k_chunks * kChunkBytes + dp * 16;
+            double nxA = 0.0, ntA = 0.0, nxB = 0.0, ntB = 0.0;
+            bool ok = true;
+            for (int kt = static_cast<int>(t - mb * kt2); t < seg_end; ++t, ++kt) {
+                if (!warp_wait(&full[stage], phase, err)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* sX = smem + stage * stage_bytes;
+                const uint4 xa = *reinterpret_cast<const uint4*>(sX + offA);
+                const uint4 xb = *reinterpret_cast<const uint4*>(sX + offB);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                // rank each group once: metadata, kept entries and the energies
+                const GroupKeys g0 = rank_group(xa.x, xa.y), g1 = rank_group(xa.z, xa.w);
+                const GroupKeys g2 = rank_group(xb.x, xb.y), g3 = rank_group(xb.z, xb.w);
+                uint2 ka, kb;
+                const uint32_t na = pick_kept(g0, xa.x, xa.y, ka.x) | (pick_kept(g1, xa.z, xa.w, ka.y) << 4);
+                const uint32_t nb = pick_kept(g2, xb.x, xb.y, kb.x) | (pick_kept(g3, xb.z, xb.w, kb.y) << 4);
+                const bool normal = group_all_normal(g0) && group_all_normal(g1) && group_all_normal(g2) &&
+                                    group_all_normal(g3);
+                if (__all_sync(0xFFFFFFFFu, normal)) {
+                    group_energy_normal(g0, nxA, ntA);
+                    group_energy_normal(g1, nxA, ntA);
+                    group_energy_normal(g2, nxB, ntB);
+                    group_energy_normal(g3, nxB, ntB);
+                } else {  // zero or subnormal entries somewhere in the warp's tile (rare)
+                    double2 e = group_energy_any(g0.k1, g0.k2, g0.k3, g0.k4);
+                    nxA += e.x;
+                    ntA += e.y;
+                    e = group_energy_any(g1.k1, g1.k2, g1.k3, g1.k4);
+                    nxA += e.x;
+                    ntA += e.y;
+                    e = group_energy_any(g2.k1, g2.k2, g2.k3, g2.k4);
+                    nxB += e.x;
+                    ntB += e.y;
+                    e = group_energy_any(g3.k1, g3.k2, g3.k3, g3.k4);
+                    nxB += e.x;
+                    ntB += e.y;
+                }
+                *reinterpret_cast<uint2*>(vA + kt * 32) = ka;
+                *reinterpret_cast<uint2*>(vB + kt * 32) = kb;
+                // metadata word: bytes (rA, u even), (rA, u odd), (rB, u even), (rB, u odd)
+                const uint32_t mine = na | (nb << 8);
+                const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
+                if (even)
+                    *reinterpret_cast<uint32_t*>(mrow + (kt >> 1) * kChunkBytes + (2 * (kt & 1) + (u >> 2)) * 4) =
+                        __byte_perm(mine, other, 0x5140);
+            }
+            if (!ok) break;
+            // the token's totals over the eight units, in a fixed order
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                nxA += __shfl_xor_sync(0xFFFFFFFFu, nxA, o);
+                ntA += __shfl_xor_sync(0xFFFFFFFFu, ntA, o);
+                nxB += __shfl_xor_sync(0xFFFFFFFFu, nxB, o);
+                ntB += __shfl_xor_sync(0xFFFFFFFFu, ntB, o);
+            }
+            if (u == 0) {
+                double* pn = a.part_norm + (seg * a.M_pad + growA) * 2;
+                pn[0] = nxA;
+                pn[1] = ntA;
+                pn[16] = nxB;  // row rB = rA + 8
+                pn[17] = ntB;
+            }
+            if (drain) {
+                const uint32_t b = n & 1u;
+                if (!warp_wait(&tfull[b], (n >> 1) & 1u, err)) break;
+                tc_fence_after();
+                const int q = warp & 3;
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * a.R_pad);
+                float* pt = a.part_T + (seg * a.M_pad + mb * kBM + q * 32 + lane) * a.R_pad;
+                for (int c = 0; c < a.R_pad; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        *reinterpret_cast<float4*>(pt + c + 4 * q4) =
+                            make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                        __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[b]);
+            }
+            ++n;
         }
     }
 
+    __syncwarp();
+    tc_fence_before();
     __syncthreads();
-    if (warp == 0 && lane == 0) {
-        for (int q = *consumed_holder; q < issued; ++q)
-            mbar_wait(&full[q % kNormStages], (q / kNormStages) & 1, nullptr);
-    }
     if (LORA && warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, tmem_cols);
@@ -202,71 +329,71 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 }
 
 // ---------------------------------------------------------------- pass 2
-struct CompressArgs {
-    int M, K;
-    int64_t M_pad, Kc_pad;
-    int k_chunks, nsplit;
+struct ScaleArgs {
+    int64_t M_pad, Kc_pad, total_tiles, grid;
+    int kt2, R_pad;
     const double* part_norm;
+    const float* part_T;
     uint16_t* vals;
-    uint8_t* meta;
     float* s_out;
+    uint16_t* T;
 };
 
-__global__ void __launch_bounds__(256) rtlynx_compress_kernel(const uint16_t* __restrict__ X, const CompressArgs a) {
-    const int warp = threadIdx.x >> 5;
+__global__ void __launch_bounds__(256) rtlynx_scale_kernel(const ScaleArgs a) {
+    constexpr int kU = 8;  // 16-byte vectors in flight per lane
     const int lane = threadIdx.x & 31;
-    const int m0 = warp, m1 = lane >> 4, p = lane & 15;
-    const int64_t slab = blockIdx.x;
-    const int64_t mb = slab >> 3;
-    const int m2 = static_cast<int>(slab & 7);
-    const int64_t row = slab * 16 + m1 * 8 + m0;
-    const int64_t k = static_cast<int64_t>(blockIdx.y) * 256 + p * 16;
-    const int64_t kc = k >> 7;
-    const bool chunk_ok = kc < a.k_chunks;
-
-    float s = 0.f;
-    if (row < a.M) {
-        double nx = 0.0, nt = 0.0;
-        for (int j = 0; j < a.nsplit; ++j) {
-            const double* pn = a.part_norm + (static_cast<int64_t>(j) * a.M_pad + row) * 2;
-            nx += pn[0];
-            nt += pn[1];
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= a.M_pad) return;
+    const int64_t first = (row / kBM) * a.kt2;
+    const int64_t c0 = stream_owner_dev(first, a.total_tiles, a.grid);
+    const int nseg = static_cast<int>(stream_owner_dev(first + a.kt2 - 1, a.total_tiles, a.grid) - c0 + 1);
+    // the first value vectors are loaded before s is formed
+    uint4* v = reinterpret_cast<uint4*>(a.vals + row * a.Kc_pad);
+    const int n16 = static_cast<int>(a.Kc_pad / 8);
+    uint4 q[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+        if (lane + 32 * u < n16) q[u] = v[lane + 32 * u];
+    // T needs no s: its partials are summed while the value loads are in flight
+    for (int c = 2 * lane; c < a.R_pad; c += 64) {
+        float t0 = 0.f, t1 = 0.f;
+        for (int j = 0; j < nseg; ++j) {
+            const float2 p = *reinterpret_cast<const float2*>(a.part_T + (j * a.M_pad + row) * a.R_pad + c);
+            t0 += p.x;
+            t1 += p.y;
         }
-        s = static_cast<float>(sqrt(nx) / (sqrt(nt) + 1e-8));
+        *reinterpret_cast<__nv_bfloat162*>(a.T + row * a.R_pad + c) = __floats2bfloat162_rn(t0, t1);
     }
-    uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-    if (row < a.M && chunk_ok) {
-        const uint16_t* xr = X + row * a.K;
-        if (k < a.K) lo = *reinterpret_cast<const uint4*>(xr + k);
-        if (k + 8 < a.K) hi = *reinterpret_cast<const uint4*>(xr + k + 8);
+    // partial sums, one segment per lane, added in segment order (every lane
+    // forms the same s)
+    double nx = 0.0, nt = 0.0;
+    for (int j0 = 0; j0 < nseg; j0 += 32) {
+        double2 part = make_double2(0.0, 0.0);
+        if (j0 + lane < nseg) part = *reinterpret_cast<const double2*>(a.part_norm + ((j0 + lane) * a.M_pad + row) * 2);
+        const int m = nseg - j0 < 32 ? nseg - j0 : 32;
+        for (int j = 0; j < m; ++j) {
+            nx += __shfl_sync(0xFFFFFFFFu, part.x, j);
+            nt += __shfl_sync(0xFFFFFFFFu, part.y, j);
+        }
     }
-    uint4 out;
-    uint32_t nib = 0;
-    nib |= compress_group(lo.x, lo.y, s, out.x);
-    nib |= compress_group(lo.z, lo.w, s, out.y) << 4;
-    nib |= compress_group(hi.x, hi.y, s, out.z) << 8;
-    nib |= compress_group(hi.z, hi.w, s, out.w) << 12;
-    if (chunk_ok && (k >> 1) < a.Kc_pad)
-        *reinterpret_cast<uint4*>(a.vals + row * a.Kc_pad + (k >> 1)) = out;
-    const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, nib, 16);
-    if (m1 == 0 && chunk_ok) {
-        const int kk = static_cast<int>(k & 127);
-        const int k2 = kk >> 5, k1 = (kk >> 4) & 1;
-        const int dp = m0 + 8 * k1 + 16 * m2;
-        uint32_t* w = reinterpret_cast<uint32_t*>(a.meta + (mb * a.k_chunks + kc) * kChunkBytes + dp * 16 + k2 * 4);
-        *w = (nib & 0xFFFFu) | (partner << 16);
-    }
-    if (blockIdx.y == 0 && p == 0) a.s_out[row] = s;
-}
-
-// ---------------------------------------------------------------- pass 3
-__global__ void rtlynx_finalize_T_kernel(const float* __restrict__ part_T, uint16_t* __restrict__ T, int64_t n,
-                                         int64_t split_stride, int nsplit) {
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float acc = 0.f;
-        for (int j = 0; j < nsplit; ++j) acc += part_T[j * split_stride + i];
-        T[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+    const float s = static_cast<float>(sqrt(nx) / (sqrt(nt) + 1e-8));
+    if (lane == 0) a.s_out[row] = s;
+    for (int i0 = lane;;) {
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (i0 + 32 * u < n16) {
+                q[u].x = scale_pair(s, q[u].x);
+                q[u].y = scale_pair(s, q[u].y);
+                q[u].z = scale_pair(s, q[u].z);
+                q[u].w = scale_pair(s, q[u].w);
+                v[i0 + 32 * u] = q[u];
+            }
+        }
+        i0 += 32 * kU;
+        if (i0 >= n16) break;
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            if (i0 + 32 * u < n16) q[u] = v[i0 + 32 * u];
     }
 }
 
@@ -302,8 +429,8 @@ __global__ void rtlynx_unpack_kernel(const Dims d, const uint16_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------- launchers
-int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
-                           cudaStream_t stream) {
+int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
+                    cudaStream_t stream) {
     const bool lora = d.R > 0 && L_B != nullptr;
     CUtensorMap tmX, tmLB;
     int rc = encode_tmap_bf16_2d(&tmX, X, d.K, d.M, d.K * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -315,52 +442,51 @@ int launch_norms_lora_down(const Dims& d, const void* X, const void* L_B, const 
     } else {
         tmLB = tmX;
     }
-    NormArgs a;
-    a.M = static_cast<int>(d.M);
+    StreamArgs a;
     a.M_pad = d.M_pad;
-    a.k_tiles = static_cast<int>(d.k_tiles);
-    a.tiles_per_split = static_cast<int>((d.k_tiles + d.nsplit - 1) / d.nsplit);
+    a.Kc_pad = d.Kc_pad;
+    a.total_tiles = d.m_blocks * d.kt2;
+    a.grid = d.grid1;
+    a.kt2 = static_cast<int>(d.kt2);
+    a.k_chunks = static_cast<int>(d.k_chunks);
     a.R_pad = lora ? static_cast<int>(d.R_pad) : 0;
+    const int stage_bytes = stream_stage_bytes(a.R_pad);
+    a.stages = 200 * 1024 / stage_bytes < 6 ? 200 * 1024 / stage_bytes : 6;
+    a.vals = ws.vals;
+    a.meta = ws.meta;
     a.part_norm = ws.part_norm;
     a.part_T = ws.part_T;
     a.err = err;
-    const int smem = kNormStages * norm_stage_bytes(a.R_pad) + 256 + 1024;
-    dim3 grid(static_cast<unsigned>(d.m_blocks), static_cast<unsigned>(d.nsplit));
+    const int smem = a.stages * stage_bytes + 256 + 1024;
+    const dim3 grid(static_cast<unsigned>(d.grid1));
     cudaError_t e;
     if (lora) {
-        e = cudaFuncSetAttribute(rtlynx_norms_lora_down_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(rtlynx_sparsify_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem);
         if (e != cudaSuccess) return e;
-        rtlynx_norms_lora_down_kernel<true><<<grid, kNormThreads, smem, stream>>>(tmX, tmLB, a);
+        rtlynx_sparsify_stream_kernel<true><<<grid, kStreamThreads, smem, stream>>>(tmX, tmLB, a);
     } else {
-        e = cudaFuncSetAttribute(rtlynx_norms_lora_down_kernel<false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(rtlynx_sparsify_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem);
         if (e != cudaSuccess) return e;
-        rtlynx_norms_lora_down_kernel<false><<<grid, kNormThreads, smem, stream>>>(tmX, tmLB, a);
+        rtlynx_sparsify_stream_kernel<false><<<grid, kStreamThreads, smem, stream>>>(tmX, tmLB, a);
     }
     e = cudaGetLastError();
-    if (e != cudaSuccess || !lora) return e;
-    const int64_t n = d.M_pad * d.R_pad;
-    const int blocks = static_cast<int>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-    rtlynx_finalize_T_kernel<<<blocks, 256, 0, stream>>>(ws.part_T, ws.T, n, d.M_pad * d.R_pad,
-                                                          static_cast<int>(d.nsplit));
-    return cudaGetLastError();
-}
+    if (e != cudaSuccess) return e;
 
-int launch_compress(const Dims& d, const void* X, const Workspace& ws, cudaStream_t stream) {
-    CompressArgs a;
-    a.M = static_cast<int>(d.M);
-    a.K = static_cast<int>(d.K);
-    a.M_pad = d.M_pad;
-    a.Kc_pad = d.Kc_pad;
-    a.k_chunks = static_cast<int>(d.k_chunks);
-    a.nsplit = static_cast<int>(d.nsplit);
-    a.part_norm = ws.part_norm;
-    a.vals = ws.vals;
-    a.meta = ws.meta;
-    a.s_out = ws.s;
-    dim3 grid(static_cast<unsigned>(d.M_pad / 16), static_cast<unsigned>((d.k_chunks * kChunkK + 255) / 256));
-    rtlynx_compress_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(X), a);
+    ScaleArgs b;
+    b.M_pad = d.M_pad;
+    b.Kc_pad = d.Kc_pad;
+    b.total_tiles = a.total_tiles;
+    b.grid = d.grid1;
+    b.kt2 = a.kt2;
+    b.R_pad = a.R_pad;
+    b.part_norm = ws.part_norm;
+    b.part_T = ws.part_T;
+    b.vals = ws.vals;
+    b.s_out = ws.s;
+    b.T = ws.T;
+    rtlynx_scale_kernel<<<static_cast<unsigned>(d.M_pad / 8), 256, 0, stream>>>(b);
     return cudaGetLastError();
 }
 

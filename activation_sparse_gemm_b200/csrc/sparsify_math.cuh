@@ -1,9 +1,9 @@
 // Per-group arithmetic of the RT-Lynx sparsify step (RT-Lynx summary page,
-// four-step pipeline paragraph, step 1), shared by the prologue kernels.
+// four-step pipeline paragraph, step 1), used by the prologue kernels.
 //
 // A group is four consecutive bf16 entries held in two 32-bit words.  The
 // 2-of-4 rule keeps the two largest magnitudes, equal magnitudes going to the
-// lower index.  Both prologue passes rank the group by the unique key
+// lower index.  The prologue ranks each group by the unique key
 // (|x| bits << 2) | (3 - index): integer order of the keys is magnitude order
 // with the lower index winning ties, so the two largest keys are the kept
 // entries.
@@ -34,41 +34,48 @@ __device__ __forceinline__ GroupKeys rank_group(uint32_t w01, uint32_t w23) {
     return g;
 }
 
-// |x| of a key as a float (exact).
-__device__ __forceinline__ float key_mag(uint32_t key) { return __uint_as_float((key >> 2) << 16); }
-
 // A normal bf16 magnitude (exponent field 1..254) as a double, built from its
 // bits: same significand, exponent rebiased from 127 to 1023.  Exact.
 __device__ __forceinline__ double bf16_mag_to_double(uint32_t mag15) {
     return __hiloint2double(static_cast<int>((mag15 << 13) + ((1023u - 127u) << 20)), 0);
 }
 
-// Adds sum(x^2) and the sum of the two largest squares of one group to the
-// token's double accumulators.  Products of bf16 values are exact in double
-// and each fused multiply-add rounds once, so the sums carry double rounding
-// only.  Zero and subnormal entries take the (rare) converting path.
-__device__ __forceinline__ void group_energy(uint32_t w01, uint32_t w23, double& all, double& kept) {
-    const uint32_t m0 = w01 & 0x7FFFu, m1 = (w01 >> 16) & 0x7FFFu;
-    const uint32_t m2 = w23 & 0x7FFFu, m3 = (w23 >> 16) & 0x7FFFu;
-    const uint32_t h01 = max(m0, m1), l01 = min(m0, m1), h23 = max(m2, m3), l23 = min(m2, m3);
-    const uint32_t mh = min(h01, h23), ml = max(l01, l23);
-    const uint32_t t1 = max(h01, h23), t2 = max(mh, ml);  // kept: the two largest
-    const uint32_t t3 = min(mh, ml), t4 = min(l01, l23);  // dropped
-    double e1, e2, e3, e4;
-    if (t4 >= 0x80u) {
-        e1 = bf16_mag_to_double(t1);
-        e2 = bf16_mag_to_double(t2);
-        e3 = bf16_mag_to_double(t3);
-        e4 = bf16_mag_to_double(t4);
-    } else {  // zero or subnormal entries
-        e1 = __uint_as_float(t1 << 16);
-        e2 = __uint_as_float(t2 << 16);
-        e3 = __uint_as_float(t3 << 16);
-        e4 = __uint_as_float(t4 << 16);
-    }
+// The metadata nibble i0 | (i1 << 2) of a ranked group (i0 < i1, the kept
+// indices), and its two kept entries, unscaled, packed as bf16x2 (i0 in the
+// low half).
+__device__ __forceinline__ uint32_t pick_kept(const GroupKeys& g, uint32_t w01, uint32_t w23, uint32_t& kept) {
+    const uint32_t ia = (~g.k1) & 3u, ib = (~g.k2) & 3u;  // 3 - (key & 3)
+    const uint32_t i0 = min(ia, ib), i1 = max(ia, ib);
+    // byte selector picking half-words i0 and i1 out of {w01, w23}
+    const uint32_t sel = (i0 * 0x22u + 0x10u) | ((i1 * 0x22u + 0x10u) << 8);
+    kept = __byte_perm(w01, w23, sel);
+    return i0 | (i1 << 2);
+}
+
+// True when the smallest entry of the group is a normal number (so are the others).
+__device__ __forceinline__ bool group_all_normal(const GroupKeys& g) { return g.k4 >= (0x80u << 2); }
+
+// Adds sum(x^2) of a ranked group whose entries are all normal numbers to
+// `all` and the sum of its two largest squares to `top`.  Each entry is
+// rebuilt as a double from its bits; products of bf16 values are exact in
+// double and each fused multiply-add rounds once.
+__device__ __forceinline__ void group_energy_normal(const GroupKeys& g, double& all, double& top) {
+    const double e1 = bf16_mag_to_double(g.k1 >> 2), e2 = bf16_mag_to_double(g.k2 >> 2);
+    const double e3 = bf16_mag_to_double(g.k3 >> 2), e4 = bf16_mag_to_double(g.k4 >> 2);
     const double k = fma(e2, e2, e1 * e1);
-    kept += k;
+    top += k;
     all += fma(e4, e4, fma(e3, e3, k));
+}
+
+// The same sums for a group that may hold zero or subnormal entries (they go
+// through float, which holds every bf16 value exactly).  Kept out of line:
+// it runs only for the rare tiles that need it, so the common path never pays
+// for its conversions.  Returns (sum of all four squares, sum of the top two).
+static __device__ __noinline__ double2 group_energy_any(uint32_t k1, uint32_t k2, uint32_t k3, uint32_t k4) {
+    const double e1 = __uint_as_float((k1 >> 2) << 16), e2 = __uint_as_float((k2 >> 2) << 16);
+    const double e3 = __uint_as_float((k3 >> 2) << 16), e4 = __uint_as_float((k4 >> 2) << 16);
+    const double k = fma(e2, e2, e1 * e1);
+    return make_double2(fma(e4, e4, fma(e3, e3, k)), k);
 }
 
 // bf16 nearest-even of the exact product s*x (one rounding, like the
@@ -102,17 +109,10 @@ __device__ __forceinline__ uint32_t mul_round_bf16x2(float s, float x0, float x1
     return packed;
 }
 
-// One group: returns the metadata nibble i0 | (i1 << 2) (i0 < i1, the kept
-// indices) and the two kept values, rounded s*x, packed as bf16x2 (i0 low).
-__device__ __forceinline__ uint32_t compress_group(uint32_t w01, uint32_t w23, float s, uint32_t& packed) {
-    const GroupKeys g = rank_group(w01, w23);
-    const uint32_t ia = (~g.k1) & 3u, ib = (~g.k2) & 3u;  // 3 - (key & 3)
-    const uint32_t i0 = min(ia, ib), i1 = max(ia, ib);
-    // byte selector picking half-words i0 and i1 out of {w01, w23}
-    const uint32_t sel = (i0 * 0x22u + 0x10u) | ((i1 * 0x22u + 0x10u) << 8);
-    const uint32_t xx = __byte_perm(w01, w23, sel);
-    packed = mul_round_bf16x2(s, __uint_as_float(xx << 16), __uint_as_float(xx & 0xFFFF0000u));
-    return i0 | (i1 << 2);
+// Rescales a packed pair of kept bf16 entries by s: each product s*x rounded
+// once to bf16 (nearest even).
+__device__ __forceinline__ uint32_t scale_pair(float s, uint32_t packed) {
+    return mul_round_bf16x2(s, __uint_as_float(packed << 16), __uint_as_float(packed & 0xFFFF0000u));
 }
 
 }  // namespace rtlynx

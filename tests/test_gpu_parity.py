@@ -137,7 +137,7 @@ def test_sparsify_bruteforce_alphabet():
 
 
 @pytest.mark.parametrize("M,K,R", [(128, 256, 64), (1, 64, 8), (127, 72, 16), (129, 264, 32), (200, 520, 0),
-                                   (256, 3072, 64)])
+                                   (256, 3072, 64), (2000, 1000, 64), (5000, 136, 16), (128, 16384, 64)])
 def test_sparsify_small(M, K, R):
     X, _, _, L_B = make_custom(M, K, 16, R if R else 8, seed=200 + M)
     frac_same = check_sparsify(X, L_B if R else None)
@@ -178,7 +178,8 @@ def test_sparsify_raw_workspace_layout():
 
 # ------------------------------------------------------------------ the fused layer
 @pytest.mark.parametrize("M,K,N,R", [(128, 256, 256, 64), (1, 64, 8, 8), (127, 72, 264, 16), (129, 264, 520, 32),
-                                     (300, 512, 256, 0), (256, 1024, 512, 256), (384, 3072, 768, 64)])
+                                     (300, 512, 256, 0), (256, 1024, 512, 256), (384, 3072, 768, 64),
+                                     (2000, 1000, 136, 64), (5000, 136, 264, 16), (128, 16384, 72, 64)])
 def test_sparse_linear_small(M, K, N, R):
     X, W, L_A, L_B = make_custom(M, K, N, R if R else 8, seed=300 + M)
     if R == 0:
