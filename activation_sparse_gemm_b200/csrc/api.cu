@@ -147,6 +147,30 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
     // run holds at least L = floor(total / grid1) tiles.
     const int64_t run = total / d.grid1;
     d.max_segs = (d.kt2 - 2) / run + 2;
+    // Sparse GEMM: full rounds of tiles over the pairs, then the remainder
+    // tiles cut along K so that every pair has a part (3 to kMaxSplit parts a
+    // tile, each at least two stages long).
+    const int64_t m_pairs = d.M_pad / (2 * kBM);
+    const int64_t n_tiles = (N + kPairBN - 1) / kPairBN;
+    d.gemm_tiles = m_pairs * n_tiles;
+    const int64_t max_pairs = (num_sms > 0 ? num_sms : 148) / 2;
+    d.gemm_pairs = d.gemm_tiles < max_pairs ? d.gemm_tiles : max_pairs;
+    const int64_t rem = d.gemm_tiles % d.gemm_pairs;
+    const int64_t n_iter = d.k_chunks + d.R_pad / 64;
+    int64_t split = rem > 0 ? d.gemm_pairs / rem : 1;
+    if (split > kMaxSplit) split = kMaxSplit;
+    if (split > n_iter / 2) split = n_iter / 2;
+    // A split tile pays for a partial store, a ticket and a fix-up; two parts
+    // save less than that costs.
+    if (split < 3) {
+        d.tail_full = d.gemm_tiles;
+        d.tail_split = 1;
+        d.tail_units = 0;
+    } else {
+        d.tail_full = d.gemm_tiles - rem;
+        d.tail_split = split;
+        d.tail_units = rem * split;
+    }
     return d;
 }
 
@@ -165,6 +189,10 @@ WsLayout make_ws_layout(const Dims& d) {
     off = align256(off + static_cast<size_t>(d.max_segs) * d.M_pad * 2 * 8);
     l.part_T = off;
     off = align256(off + static_cast<size_t>(d.max_segs) * d.M_pad * d.R_pad * 4);
+    l.split_part = off;
+    off = align256(off + static_cast<size_t>(d.tail_units) * 2 * kSplitSlotFloats * 4);
+    l.split_cnt = off;
+    off = align256(off + static_cast<size_t>(d.gemm_tiles - d.tail_full) * 2 * 4);
     l.total = off;
     return l;
 }
@@ -178,6 +206,8 @@ Workspace carve(void* base, const WsLayout& l) {
     w.T = reinterpret_cast<uint16_t*>(b + l.T);
     w.part_norm = reinterpret_cast<double*>(b + l.part_norm);
     w.part_T = reinterpret_cast<float*>(b + l.part_T);
+    w.split_part = reinterpret_cast<float*>(b + l.split_part);
+    w.split_cnt = reinterpret_cast<int*>(b + l.split_cnt);
     return w;
 }
 

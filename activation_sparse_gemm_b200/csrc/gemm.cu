@@ -80,13 +80,61 @@ struct PairArgs {
     int k_stages;      // main-loop stages per tile (128-wide K chunks when sparse, 64-wide when dense)
     int lora_stages;   // 64-wide LoRA stages per tile
     int k_chunks;      // metadata chunks per 128-row block
+    // schedule: tiles [0, full_tiles) round-robin over the pairs; tile
+    // full_tiles + u / tail_split is cut along K, part u % tail_split going to
+    // pair u (u < tail_units)
+    int full_tiles, tail_split, tail_units;
+    float* split_part;  // fp32 partial tile of each part, per CTA of the pair
+    int* split_cnt;     // arrival ticket of each split tile, per CTA of the pair (zeroed by the prologue)
     int* err;
 };
+
+// One work item of a pair: output tile `tile` over stages [kb, ke) of its
+// k_stages + lora_stages stages; `unit` >= 0 marks a part of a split tile.
+struct PairWork {
+    int tile, kb, ke, unit;
+};
+
+__device__ __forceinline__ bool pair_work(int idx, int pair, int num_pairs, const PairArgs& a, PairWork& w) {
+    const int n_iter = a.k_stages + a.lora_stages;
+    const int ndp = pair < a.full_tiles ? (a.full_tiles - pair + num_pairs - 1) / num_pairs : 0;
+    if (idx < ndp) {
+        w.tile = pair + idx * num_pairs;
+        w.kb = 0;
+        w.ke = n_iter;
+        w.unit = -1;
+        return true;
+    }
+    if (idx == ndp && pair < a.tail_units) {
+        const int j = pair % a.tail_split;
+        w.tile = a.full_tiles + pair / a.tail_split;
+        w.kb = j * n_iter / a.tail_split;
+        w.ke = (j + 1) * n_iter / a.tail_split;
+        w.unit = pair;
+        return true;
+    }
+    return false;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* err) {
     uint32_t ok = 0;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err) ? 1u : 0u;
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+// One 32-column chunk of the accumulator (16 columns when `half`) into r,
+// waited for.  `half` must be the same in the whole warp.
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, bool half, uint32_t (&r)[32]) {
+    if (half) {
+        uint32_t h[16];
+        tmem_ld_32x32b_x16(taddr, h);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) r[q] = h[q];
+    } else {
+        tmem_ld_32x32b_x32(taddr, r);
+        tmem_ld_wait();
+    }
 }
 
 template <bool SPARSE, int BN>
@@ -104,7 +152,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     uint64_t* acc_full = empty + G::STAGES;   // [2]
     uint64_t* acc_empty = acc_full + 2;       // [2], used in the leader only
     uint64_t* done_bar = acc_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done_bar + 1);
+    uint64_t* epi_done = done_bar + 1;  // split tile: the four epilogue warps stored their partials
+    uint64_t* epi_dec = epi_done + 1;   // split tile: the ticket has been read
+    uint64_t* fix_full = epi_dec + 1;   // [8] split fix-up: a chunk of the other parts has landed
+    uint64_t* fix_empty = fix_full + 8; // [8] split fix-up: the four epilogue warps are done with it
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(fix_empty + 8);
+    uint32_t* epi_last = tmem_holder + 1;  // split tile: this CTA sums the parts
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -124,6 +177,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA of the pair
         }
         mbar_init(done_bar, 1);
+        mbar_init(epi_done, 4);
+        mbar_init(epi_dec, 1);
+        for (int b = 0; b < 8; ++b) {
+            mbar_init(&fix_full[b], 1);
+            mbar_init(&fix_empty[b], 4);
+        }
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
@@ -145,8 +204,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_base = *tmem_holder;
     const uint32_t tmem_meta = tmem_base + 2 * BN;
 
-    const int num_tiles = args.m_pairs * args.n_tiles;
-    const int total_k = args.k_stages + args.lora_stages;
+    PairWork w;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -154,13 +212,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                const int mp = tile % args.m_pairs;
-                const int nt = tile / args.m_pairs;
+            for (int idx = 0; ok && pair_work(idx, pair, num_pairs, args, w); ++idx) {
+                const int mp = w.tile % args.m_pairs;
+                const int nt = w.tile / args.m_pairs;
                 const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM;
                 const int col0 = nt * BN + static_cast<int>(rank) * G::BN_HALF;
                 const int chunk0 = (row0 / kBM) * args.k_chunks;
-                for (int kt = 0; kt < total_k; ++kt) {
+                for (int kt = w.kb; kt < w.ke; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, err)) {
                         ok = false;
                         break;
@@ -216,9 +274,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint64_t off = 0;  // stage offset in 16-byte units
-            int local = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+            for (int local = 0; ok && pair_work(local, pair, num_pairs, args, w); ++local) {
                 const int buf = local & 1;
                 const uint32_t use = static_cast<uint32_t>(local >> 1);
                 if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, err)) {
@@ -227,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
-                for (int kt = 0; kt < total_k; ++kt) {
+                for (int kt = w.kb; kt < w.ke; ++kt) {
                     if (!mbar_wait(&full[stage], phase, err)) {
                         ok = false;
                         break;
@@ -235,8 +292,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     tc_fence_after();
                     const uint64_t a = descA0 + off;
                     const uint64_t b = descB0 + off;
+                    const uint32_t acc = kt != w.kb;  // the item's first stage starts the accumulator
                     if (kt < args.k_stages) {
-                        const uint32_t acc = kt != 0;
                         if constexpr (SPARSE) {
                             tmem_cp_128x128b_pair(tmem_meta, descE0 + off);
                             mma_sp_f16_pair(d, a, b, e01, id0, acc);
@@ -250,7 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                             mma_f16_pair(d, a + 6, b + 6, idesc_main, 1u);
                         }
                     } else {
-                        mma_f16_pair(d, a, b, idesc_dense, 1u);
+                        mma_f16_pair(d, a, b, idesc_dense, acc);
                         mma_f16_pair(d, a + 2, b + 2, idesc_dense, 1u);
                         mma_f16_pair(d, a + 4, b + 4, idesc_dense, 1u);
                         mma_f16_pair(d, a + 6, b + 6, idesc_dense, 1u);
@@ -273,68 +330,175 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     } else {
         const int quad = warp & 3;  // warps 2..5 own tensor-memory lane quadrants 2,3,0,1
         const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+        const int row_in_cta = quad * 32 + lane;
         uint8_t* stage_buf = epi + (warp - 2) * 2 * kEpiBufBytes;
         int sbuf = 0;
-        int local = 0;
-        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
+        for (int local = 0; pair_work(local, pair, num_pairs, args, w); ++local) {
             const int buf = local & 1;
             const uint32_t use = static_cast<uint32_t>(local >> 1);
             if (!warp_wait(&acc_full[buf], use & 1u, err)) break;
             tc_fence_after();
-            const int mp = tile % args.m_pairs;
-            const int nt = tile / args.m_pairs;
+            const int mp = w.tile % args.m_pairs;
+            const int nt = w.tile / args.m_pairs;
             const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM + quad * 32;
             const int col0 = nt * BN;
             const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN) + lane_addr;
+            const bool split = w.unit >= 0;
+            bool write_y = true;
+            const int S = args.tail_split;
+            const int tt = w.tile - args.full_tiles;  // index among the split tiles
+            const int my_j = split ? w.unit % S : 0;
+            // fp32 partial slot of part j of this split tile, this CTA's half
+            auto slot = [&](int j) {
+                return args.split_part + (static_cast<size_t>(tt * S + j) * 2 + rank) * kSplitSlotFloats;
+            };
+            // Fix-up buffers: the pipeline stages, idle once the accumulator of
+            // the pair's last work item (the split part) is complete.  They
+            // form a ring of `nslot` slots; slot b holds chunk c (c % nslot ==
+            // b) of the S - 1 other parts, 16 KB each.  With two parts every
+            // chunk has its own slot and all of them are requested at once.
+            constexpr uint32_t kFixChunk = kBM * 32 * 4;
+            constexpr int kChunks = (BN + 31) / 32;
+            const int per_slot = (S > 1 ? S - 1 : 1) * static_cast<int>(kFixChunk);
+            int nslot = (G::STAGES * G::STAGE_BYTES) / per_slot;
+            nslot = nslot < kChunks ? nslot : kChunks;
+            auto fix_issue = [&](int c) {  // one thread
+                const int b = c % nslot;
+                uint8_t* dst = smem + b * per_slot;
+                const uint32_t bytes = (BN - c * 32) < 32 ? kFixChunk / 2 : kFixChunk;
+                mbar_arrive_expect_tx(&fix_full[b], bytes * static_cast<uint32_t>(S - 1));
+                for (int j = 0, jj = 0; j < S; ++j) {
+                    if (j == my_j) continue;
+                    bulk_load(dst + jj * kFixChunk, slot(j) + c * (kFixChunk / 4), bytes, &fix_full[b]);
+                    ++jj;
+                }
+            };
+            if (split) {
+                // This CTA's fp32 partial goes to its slot; the last of the
+                // tile's parts to arrive sums all of them in part order.
+                float* own = slot(my_j);
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                const bool half = (BN - c) < 32;  // 16-column tail chunk
-                uint32_t r[32];
-                if (half) {
-                    uint32_t h[16];
-                    tmem_ld_32x32b_x16(acc + static_cast<uint32_t>(c), h);
-                    tmem_ld_wait();
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t r[32];
+                    const bool half = (BN - c) < 32;
+                    tmem_ld_chunk(acc + static_cast<uint32_t>(c), half, r);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) r[q] = h[q];
-                } else {
-                    tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c), r);
-                    tmem_ld_wait();
+                    for (int q = 0; q < 8; ++q)
+                        if (!half || q < 4)
+                            reinterpret_cast<float4*>(own)[((c / 32) * 8 + q) * kBM + row_in_cta] =
+                                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                            __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
                 }
-                uint8_t* sb = stage_buf + sbuf * kEpiBufBytes;
-                if (lane == 0) bulk_wait_group_read<1>();  // the store that last used sb has read it
+                __threadfence();
                 __syncwarp();
-                if (!half) {
-                    // 32 rows x 64 B, 64B swizzle: 16-byte unit q of row i at q ^ ((i / 2) % 4)
-                    uint8_t* row = sb + lane * 64;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-                        pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-                        pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-                        pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-                        *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) = pk;
+                if (lane == 0) mbar_arrive(epi_done);
+                if (warp == 2) {
+                    const bool stored = warp_wait(epi_done, 0, err);
+                    if (lane == 0) {
+                        uint32_t last = 0;
+                        if (stored) {
+                            const int old = atomicAdd(&args.split_cnt[tt * 2 + rank], 1);
+                            last = old == S - 1;
+                            if (last) {
+                                __threadfence();
+                                args.split_cnt[tt * 2 + rank] = 0;
+                                for (int c = 0; c < nslot; ++c) fix_issue(c);
+                            }
+                        }
+                        *epi_last = last;
+                        mbar_arrive(epi_dec);
                     }
-                } else {
-                    // 32 rows x 32 B, 32B swizzle: 16-byte unit q of row i at q ^ ((i / 4) % 2)
-                    uint8_t* row = sb + lane * 32;
+                    __syncwarp();
+                }
+                if (!warp_wait(epi_dec, 0, err)) break;
+                write_y = *reinterpret_cast<volatile uint32_t*>(epi_last) != 0;
+            }
+            if (write_y) {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    const bool half = (BN - c) < 32;  // 16-column tail chunk
+                    const int ci = c / 32;
+                    uint32_t r[32];
+                    if (!split) {
+                        tmem_ld_chunk(acc + static_cast<uint32_t>(c), half, r);
+                    } else {
+                        const int b = ci % nslot;
+                        const uint32_t round = static_cast<uint32_t>(ci / nslot);
+                        if (!warp_wait(&fix_full[b], round & 1u, err)) break;
+                        const uint8_t* fb = smem + b * per_slot;
+                        float sum[32];
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-                        pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-                        pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-                        pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-                        *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 2) & 1)) << 4)) = pk;
+                        for (int q = 0; q < 32; ++q) sum[q] = 0.f;
+                        for (int j = 0, jj = 0; j < S; ++j) {
+                            uint32_t t[32];
+                            if (j == my_j) {
+                                tmem_ld_chunk(acc + static_cast<uint32_t>(c), half, t);
+                            } else {
+                                const float4* src = reinterpret_cast<const float4*>(fb + jj * kFixChunk);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    if (!half || q < 4) {
+                                        const float4 v = src[q * kBM + row_in_cta];
+                                        t[4 * q] = __float_as_uint(v.x);
+                                        t[4 * q + 1] = __float_as_uint(v.y);
+                                        t[4 * q + 2] = __float_as_uint(v.z);
+                                        t[4 * q + 3] = __float_as_uint(v.w);
+                                    }
+                                }
+                                ++jj;
+                            }
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (!half || q < 16) sum[q] += __uint_as_float(t[q]);
+                        }
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(sum[q]);
+                        __syncwarp();
+                        if (ci + nslot < kChunks) {  // refill this slot with chunk ci + nslot
+                            if (lane == 0) mbar_arrive(&fix_empty[b]);
+                            if (warp == 2) {
+                                const bool free_slot = warp_wait(&fix_empty[b], round & 1u, err);
+                                if (lane == 0 && free_slot) fix_issue(ci + nslot);
+                                __syncwarp();
+                            }
+                        }
                     }
+                    uint8_t* sb = stage_buf + sbuf * kEpiBufBytes;
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used sb has read it
+                    __syncwarp();
+                    if (!half) {
+                        // 32 rows x 64 B, 64B swizzle: 16-byte unit q of row i at q ^ ((i / 2) % 4)
+                        uint8_t* row = sb + lane * 64;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                            pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                            pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                            pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                            *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) = pk;
+                        }
+                    } else {
+                        // 32 rows x 32 B, 32B swizzle: 16-byte unit q of row i at q ^ ((i / 4) % 2)
+                        uint8_t* row = sb + lane * 32;
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+                            pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+                            pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+                            pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+                            *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 2) & 1)) << 4)) = pk;
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(half ? &tmY16 : &tmY, sb, col0 + c, row0);
+                        bulk_commit_group();
+                    }
+                    sbuf ^= 1;
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(half ? &tmY16 : &tmY, sb, col0 + c, row0);
-                    bulk_commit_group();
-                }
-                sbuf ^= 1;
             }
             tc_fence_before();
             __syncwarp();
@@ -373,8 +537,6 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
     kernel<<<2 * pairs, kPairThreads, G::SMEM_BYTES, stream>>>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args);
     return cudaGetLastError();
 }
-
-constexpr int kPairBN = 240;
 
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int num_sms, int* err, cudaStream_t stream) {
@@ -424,6 +586,17 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.k_stages = static_cast<int>(sparse ? d.k_chunks : d.k_tiles);
     args.lora_stages = lora ? static_cast<int>(d.R_pad / 64) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
+    if (sparse) {
+        args.full_tiles = static_cast<int>(d.tail_full);
+        args.tail_split = static_cast<int>(d.tail_split);
+        args.tail_units = static_cast<int>(d.tail_units);
+    } else {  // dense-skip has no workspace: every tile whole, round-robin
+        args.full_tiles = args.m_pairs * args.n_tiles;
+        args.tail_split = 1;
+        args.tail_units = 0;
+    }
+    args.split_part = ws.split_part;
+    args.split_cnt = ws.split_cnt;
     args.err = err;
     return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
                   : launch_pair<false, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);

@@ -14,6 +14,10 @@ constexpr int kBN = 256;          // output columns per tile
 constexpr int kBK = 64;           // logical K per pipeline stage
 constexpr int kChunkK = 128;      // logical K per metadata chunk (4 sparse MMAs of K = 32)
 constexpr int kChunkBytes = 2048; // 128 lanes x 16 bytes of metadata per chunk
+constexpr int kPairBN = 240;      // output columns per GEMM tile (one CTA pair)
+// fp32 partial of one CTA's 128 x 240 tile: [32-column chunk 8][4-column group 8][row 128][4]
+constexpr int kSplitSlotFloats = 8 * kBM * 32;
+constexpr int kMaxSplit = 6;  // parts of one split tile (the fix-up holds two chunks of the others in shared memory)
 
 // Sizes derived from one problem.
 struct Dims {
@@ -27,6 +31,10 @@ struct Dims {
     int64_t kt2;          // 64-wide K tiles per row block in the prologue = 2 * k_chunks
     int64_t grid1;        // CTAs of the streaming prologue pass
     int64_t max_segs;     // most CTAs whose tile runs meet one row block (partial-sum slots)
+    // Sparse GEMM schedule: `gemm_pairs` persistent CTA pairs take the first
+    // `tail_full` tiles round-robin; each of the remaining tiles is cut along K
+    // into `tail_split` parts, one per pair (`tail_units` parts in all).
+    int64_t gemm_pairs, gemm_tiles, tail_full, tail_split, tail_units;
 };
 
 // The streaming prologue cuts the m_blocks * kt2 tiles into `grid` contiguous
@@ -39,7 +47,7 @@ __host__ __device__ inline int64_t stream_owner(int64_t t, int64_t total, int64_
 
 // Byte offsets of the sparse-mode workspace regions (each 256-byte aligned).
 struct WsLayout {
-    size_t vals, meta, s, T, part_norm, part_T, total;
+    size_t vals, meta, s, T, part_norm, part_T, split_part, split_cnt, total;
 };
 
 Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms);
@@ -52,6 +60,8 @@ struct Workspace {
     uint16_t* T;          // [M_pad, R_pad] bf16, X L_B^T
     double* part_norm;    // [max_segs, M_pad, 2] partial sums of x^2 and of kept x^2
     float* part_T;        // [max_segs, M_pad, R_pad] partial X L_B^T
+    float* split_part;    // [tail_units, 2, kSplitSlotFloats] fp32 partial tiles of the split tail
+    int* split_cnt;       // [2 * (gemm_tiles - tail_full)] arrival tickets of the split tiles
 };
 
 // Tensor-map encoding through the driver entry point (no libcuda link needed).

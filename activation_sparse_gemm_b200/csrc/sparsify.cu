@@ -47,6 +47,8 @@ struct StreamArgs {
     uint8_t* meta;
     double* part_norm;
     float* part_T;
+    int* split_cnt;  // arrival tickets of the GEMM's split tiles, zeroed here for the GEMM that follows
+    int n_split_cnt;
     int* err;
 };
 
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = LORA ? *tmem_holder : 0u;
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.n_split_cnt; i += blockDim.x) a.split_cnt[i] = 0;
 
     // Role warps run their loops with all 32 lanes (waits by every lane, the
     // single-thread actions predicated on lane 0), so every warp reaches the
@@ -456,6 +460,8 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
     a.meta = ws.meta;
     a.part_norm = ws.part_norm;
     a.part_T = ws.part_T;
+    a.split_cnt = ws.split_cnt;
+    a.n_split_cnt = static_cast<int>(2 * (d.gemm_tiles - d.tail_full));
     a.err = err;
     const int smem = a.stages * stage_bytes + 256 + 1024;
     const dim3 grid(static_cast<unsigned>(d.grid1));
