@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace rtlynx {
 
 // Tile geometry shared by the prologue and the GEMM.
@@ -73,6 +75,26 @@ inline int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inne
                                CUtensorMapSwizzle swizzle) {
     return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, row_stride_bytes, box_inner,
                           box_outer, swizzle);
+}
+
+// Launches `kernel` as a programmatic dependent of the preceding kernel in
+// the stream: it may be scheduled while that kernel drains and must call
+// grid_dependency_wait before reading what the preceding kernel wrote.
+template <typename... KArgs, typename... Args>
+int launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    return e != cudaSuccess ? static_cast<int>(e) : static_cast<int>(cudaGetLastError());
 }
 
 // Launchers; each returns a cudaError_t value (0 on success).

@@ -103,6 +103,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
 }
 
 // ---------------------------------------------------------------- TMA / bulk copies
+// Programmatic dependent launch: the kernel that follows in the stream may
+// start once every CTA of this grid has called launch_dependents (or exited);
+// grid_dependency_wait blocks until the preceding grid has completed and its
+// memory operations are visible (it returns at once when the kernel was not
+// launched as a dependent).
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = LORA ? *tmem_holder : 0u;
+    launch_dependents();  // the scale pass may be scheduled; it waits for this grid to finish
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.n_split_cnt; i += blockDim.x) a.split_cnt[i] = 0;
 
@@ -347,8 +348,10 @@ __global__ void __launch_bounds__(256) rtlynx_scale_kernel(const ScaleArgs a) {
     constexpr int kU = 8;  // 16-byte vectors in flight per lane
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (row >= a.M_pad) return;
     const int64_t first = (row / kBM) * a.kt2;
+    grid_dependency_wait();  // everything pass 1 wrote is visible from here on
+    launch_dependents();
+    if (row >= a.M_pad) return;
     const int64_t c0 = stream_owner_dev(first, a.total_tiles, a.grid);
     const int nseg = static_cast<int>(stream_owner_dev(first + a.kt2 - 1, a.total_tiles, a.grid) - c0 + 1);
     // the first value vectors are loaded before s is formed
@@ -492,8 +495,7 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
     b.vals = ws.vals;
     b.s_out = ws.s;
     b.T = ws.T;
-    rtlynx_scale_kernel<<<static_cast<unsigned>(d.M_pad / 8), 256, 0, stream>>>(b);
-    return cudaGetLastError();
+    return launch_dependent(rtlynx_scale_kernel, dim3(static_cast<unsigned>(d.M_pad / 8)), dim3(256), 0, stream, b);
 }
 
 int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,
