@@ -77,6 +77,7 @@ struct PairShape {
 struct PairArgs {
     int M, N;
     int m_pairs, n_tiles;
+    int group_n;       // column tiles per raster group (see tile_coords)
     int k_stages;      // main-loop stages per tile (128-wide K chunks when sparse, 64-wide when dense)
     int lora_stages;   // 64-wide LoRA stages per tile
     int k_chunks;      // metadata chunks per 128-row block
@@ -88,6 +89,20 @@ struct PairArgs {
     int* split_cnt;     // arrival ticket of each split tile, per CTA of the pair (zeroed by the prologue)
     int* err;
 };
+
+// Raster order of the tiles: column tiles are taken in groups of group_n; a
+// group's tiles are numbered row pair by row pair, so a wave of consecutive
+// tiles covers a few row pairs across group_n column tiles, and the group's
+// slice of W stays in L2 while all row pairs sweep past it.  The last group
+// may be narrower.
+__device__ __forceinline__ void tile_coords(int tile, const PairArgs& a, int& mp, int& nt) {
+    const int per_group = a.m_pairs * a.group_n;
+    const int g = tile / per_group;
+    const int width = min(a.group_n, a.n_tiles - g * a.group_n);
+    const int local = tile - g * per_group;
+    mp = local / width;
+    nt = g * a.group_n + local % width;
+}
 
 // One work item of a pair: output tile `tile` over stages [kb, ke) of its
 // k_stages + lora_stages stages; `unit` >= 0 marks a part of a split tile.
@@ -216,8 +231,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int idx = 0; ok && pair_work(idx, pair, num_pairs, args, w); ++idx) {
-                const int mp = w.tile % args.m_pairs;
-                const int nt = w.tile / args.m_pairs;
+                int mp, nt;
+                tile_coords(w.tile, args, mp, nt);
                 const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM;
                 const int col0 = nt * BN + static_cast<int>(rank) * G::BN_HALF;
                 const int chunk0 = (row0 / kBM) * args.k_chunks;
@@ -341,8 +356,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const uint32_t use = static_cast<uint32_t>(local >> 1);
             if (!warp_wait(&acc_full[buf], use & 1u, err)) break;
             tc_fence_after();
-            const int mp = w.tile % args.m_pairs;
-            const int nt = w.tile / args.m_pairs;
+            int mp, nt;
+            tile_coords(w.tile, args, mp, nt);
             const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM + quad * 32;
             const int col0 = nt * BN;
             const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN) + lane_addr;
@@ -592,6 +607,21 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.k_stages = static_cast<int>(sparse ? d.k_chunks : d.k_tiles);
     args.lora_stages = lora ? static_cast<int>(d.R_pad / 64) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
+    {
+        // While both operands fit in L2 (126 MB) the row-pair-fastest order
+        // (group width 1) serves each W tile to many pairs of one wave.  When
+        // they do not, column tiles are grouped so that a group's W slice,
+        // about 48 MiB, stays in L2 while the row pairs sweep past it.
+        const double a_bytes = static_cast<double>(d.M_pad) * static_cast<double>(d.K) * (sparse ? 1.125 : 2.0);
+        const double w_bytes = static_cast<double>(d.N) * static_cast<double>(d.K) * 2.0;
+        int gn = 1;
+        if (a_bytes + w_bytes > 192.0 * (1 << 20)) {
+            const double w_tile_bytes = static_cast<double>(BN) * static_cast<double>(d.K) * 2.0;
+            gn = static_cast<int>((48.0 * (1 << 20)) / w_tile_bytes);
+            gn = gn < 1 ? 1 : (gn > args.n_tiles ? args.n_tiles : gn);
+        }
+        args.group_n = gn;
+    }
     if (sparse) {
         args.full_tiles = static_cast<int>(d.tail_full);
         args.tail_split = static_cast<int>(d.tail_split);
