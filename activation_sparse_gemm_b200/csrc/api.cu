@@ -111,11 +111,46 @@ bool ensure_tmap_encoder() {
     return true;
 }
 
+namespace {
+
+// A layer call encodes the same handful of tensor maps every time it runs on
+// the same buffers; encoding is host work that can leave the GPU waiting.
+// Each host thread keeps the last kTmapCacheSize maps it encoded, keyed by
+// every argument of the encode, and hands back an identical copy.
+struct TmapKey {
+    const void* base;
+    uint64_t inner, outer, stride;
+    uint32_t box_inner, box_outer;
+    int dtype, swizzle;
+    bool operator==(const TmapKey& o) const {
+        return base == o.base && inner == o.inner && outer == o.outer && stride == o.stride &&
+               box_inner == o.box_inner && box_outer == o.box_outer && dtype == o.dtype && swizzle == o.swizzle;
+    }
+};
+constexpr int kTmapCacheSize = 16;
+struct TmapCache {
+    TmapKey key[kTmapCacheSize];
+    CUtensorMap map[kTmapCacheSize];
+    int count = 0, next = 0;
+};
+thread_local TmapCache t_tmap_cache;
+
+}  // namespace
+
 int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                    CUtensorMapSwizzle swizzle) {
     (void)elem_bytes;
     if (!g_encode) return cudaErrorInitializationError;
+    const TmapKey key{base, inner, outer, row_stride_bytes, box_inner, box_outer, static_cast<int>(dtype),
+                      static_cast<int>(swizzle)};
+    TmapCache& c = t_tmap_cache;
+    for (int i = 0; i < c.count; ++i) {
+        if (c.key[i] == key) {
+            *map = c.map[i];
+            return 0;
+        }
+    }
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_stride_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
@@ -123,7 +158,12 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, 
     CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
+    if (r != CUDA_SUCCESS) return static_cast<int>(cudaErrorInvalidValue);
+    c.key[c.next] = key;
+    c.map[c.next] = *map;
+    c.next = (c.next + 1) % kTmapCacheSize;
+    if (c.count < kTmapCacheSize) ++c.count;
+    return 0;
 }
 
 Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {

@@ -547,8 +547,9 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
                        const CUtensorMap& tmY16, const PairArgs& args, int num_sms, cudaStream_t stream) {
     using G = PairShape<SPARSE, BN>;
     auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    static std::atomic<uint64_t> smem_set{0};
+    const int e = allow_max_dynamic_smem(kernel, smem_set);
+    if (e) return e;
     const int tiles = args.m_pairs * args.n_tiles;
     const int max_pairs = num_sms / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;

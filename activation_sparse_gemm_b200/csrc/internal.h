@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace rtlynx {
@@ -95,6 +96,21 @@ int launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
     return e != cudaSuccess ? static_cast<int>(e) : static_cast<int>(cudaGetLastError());
+}
+
+// Raises `kernel`'s dynamic shared-memory limit to the most a CTA may use,
+// once per device (the attribute is kept by the runtime; setting it on every
+// launch is host work the GPU may end up waiting for).  `done` is the
+// kernel's own per-device record.
+template <typename Kernel>
+int allow_max_dynamic_smem(Kernel kernel, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return static_cast<int>(cudaErrorInvalidDevice);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return 0;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return static_cast<int>(e);
 }
 
 // Launchers; each returns a cudaError_t value (0 on success).

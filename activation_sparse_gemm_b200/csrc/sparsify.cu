@@ -469,15 +469,14 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
     const int smem = a.stages * stage_bytes + 256 + 1024;
     const dim3 grid(static_cast<unsigned>(d.grid1));
     cudaError_t e;
+    static std::atomic<uint64_t> smem_set[2];
     if (lora) {
-        e = cudaFuncSetAttribute(rtlynx_sparsify_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem);
-        if (e != cudaSuccess) return e;
+        const int rc2 = allow_max_dynamic_smem(rtlynx_sparsify_stream_kernel<true>, smem_set[1]);
+        if (rc2) return rc2;
         rtlynx_sparsify_stream_kernel<true><<<grid, kStreamThreads, smem, stream>>>(tmX, tmLB, a);
     } else {
-        e = cudaFuncSetAttribute(rtlynx_sparsify_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem);
-        if (e != cudaSuccess) return e;
+        const int rc2 = allow_max_dynamic_smem(rtlynx_sparsify_stream_kernel<false>, smem_set[0]);
+        if (rc2) return rc2;
         rtlynx_sparsify_stream_kernel<false><<<grid, kStreamThreads, smem, stream>>>(tmX, tmLB, a);
     }
     e = cudaGetLastError();
