@@ -87,6 +87,7 @@ struct PairArgs {
     int full_tiles, tail_split, tail_units;
     float* split_part;  // fp32 partial tile of each part, per CTA of the pair
     int* split_cnt;     // arrival ticket of each split tile, per CTA of the pair (zeroed by the prologue)
+    uint16_t* Y;        // [M, N] bf16 output, row-major (the dense-skip epilogue stores to it directly)
     int* err;
 };
 
@@ -149,6 +150,29 @@ __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, bool half, uint32_
     } else {
         tmem_ld_32x32b_x32(taddr, r);
         tmem_ld_wait();
+    }
+}
+
+// Rounds 32 (or 16, when `half`) fp32 values of row `row`, columns col ..,
+// to bf16 and stores them straight to Y in 16-byte pieces.  Rows >= M and
+// columns >= N (the ragged edges) are skipped; N is a multiple of 8, so every
+// 8-column piece is wholly inside or wholly outside.  Dense-skip mode writes Y
+// this way: plain stores leave the TMA unit to the producer's loads and
+// measured faster there; the sparse mode measured faster with staged TMA
+// stores.
+__device__ __forceinline__ void store_row_bf16(const PairArgs& a, int row, int col, bool half, const uint32_t (&r)[32]) {
+    if (row >= a.M) return;
+    uint4* dst = reinterpret_cast<uint4*>(a.Y + static_cast<size_t>(row) * a.N + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        if ((!half || q < 2) && col + 8 * q < a.N) {
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+            pk.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+            pk.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+            pk.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+            dst[q] = pk;
+        }
     }
 }
 
@@ -481,6 +505,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                             }
                         }
                     }
+                    if constexpr (!SPARSE) {
+                        store_row_bf16(args, row0 + lane, col0 + c, half, r);
+                        continue;
+                    }
                     uint8_t* sb = stage_buf + sbuf * kEpiBufBytes;
                     if (lane == 0) bulk_wait_group_read<1>();  // the store that last used sb has read it
                     __syncwarp();
@@ -634,6 +662,7 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     }
     args.split_part = ws.split_part;
     args.split_cnt = ws.split_cnt;
+    args.Y = static_cast<uint16_t*>(Y);
     args.err = err;
     return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
                   : launch_pair<false, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
