@@ -344,39 +344,63 @@ struct ScaleArgs {
     uint16_t* T;
 };
 
-__global__ void __launch_bounds__(256) rtlynx_scale_kernel(const ScaleArgs a) {
-    constexpr int kU = 8;  // 16-byte vectors in flight per lane
+// Eight tokens per CTA (all in one row block, so they share the segment
+// split).  Every global load the CTA needs is issued before anything waits
+// on one: the CTA's kept values (one contiguous span of 8 rows), each warp's
+// token's partial norms (one segment per lane) and partial T (up to four
+// segments at a time).  Warp w then forms token w's s and T; after one CTA
+// barrier all 256 threads rescale the span.
+__global__ void __launch_bounds__(256, 4) rtlynx_scale_kernel(const ScaleArgs a) {
+    constexpr int kRows = 8;  // tokens per CTA
+    constexpr int kU = 8;     // 16-byte value vectors in flight per thread
+    constexpr int kSegU = 4;  // partial-T segments loaded at once
+    __shared__ float s_sh[kRows];
     const int lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    const int64_t first = (row / kBM) * a.kt2;
+    const int w = threadIdx.x >> 5;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;  // M_pad is a multiple of kRows
+    const int64_t row = row0 + w;
+    const int64_t first = (row0 / kBM) * a.kt2;
     grid_dependency_wait();  // everything pass 1 wrote is visible from here on
     launch_dependents();
-    if (row >= a.M_pad) return;
     const int64_t c0 = stream_owner_dev(first, a.total_tiles, a.grid);
     const int nseg = static_cast<int>(stream_owner_dev(first + a.kt2 - 1, a.total_tiles, a.grid) - c0 + 1);
-    // the first value vectors are loaded before s is formed
-    uint4* v = reinterpret_cast<uint4*>(a.vals + row * a.Kc_pad);
+    uint4* v = reinterpret_cast<uint4*>(a.vals + row0 * a.Kc_pad);
     const int n16 = static_cast<int>(a.Kc_pad / 8);
+    const int total = kRows * n16;
     uint4 q[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u)
-        if (lane + 32 * u < n16) q[u] = v[lane + 32 * u];
-    // T needs no s: its partials are summed while the value loads are in flight
+        if (static_cast<int>(threadIdx.x) + 256 * u < total) q[u] = v[threadIdx.x + 256 * u];
+    double2 part = make_double2(0.0, 0.0);
+    if (lane < nseg) part = *reinterpret_cast<const double2*>(a.part_norm + (lane * a.M_pad + row) * 2);
+    // T needs no s: partial sums in segment order, rounded once to bf16
     for (int c = 2 * lane; c < a.R_pad; c += 64) {
         float t0 = 0.f, t1 = 0.f;
-        for (int j = 0; j < nseg; ++j) {
-            const float2 p = *reinterpret_cast<const float2*>(a.part_T + (j * a.M_pad + row) * a.R_pad + c);
-            t0 += p.x;
-            t1 += p.y;
+        for (int j0 = 0; j0 < nseg; j0 += kSegU) {
+            float2 p[kSegU];
+#pragma unroll
+            for (int j = 0; j < kSegU; ++j)
+                if (j0 + j < nseg)
+                    p[j] = *reinterpret_cast<const float2*>(a.part_T + ((j0 + j) * a.M_pad + row) * a.R_pad + c);
+#pragma unroll
+            for (int j = 0; j < kSegU; ++j) {
+                if (j0 + j < nseg) {
+                    t0 += p[j].x;
+                    t1 += p[j].y;
+                }
+            }
         }
         *reinterpret_cast<__nv_bfloat162*>(a.T + row * a.R_pad + c) = __floats2bfloat162_rn(t0, t1);
     }
-    // partial sums, one segment per lane, added in segment order (every lane
+    // partial norms, one segment per lane, added in segment order (every lane
     // forms the same s)
     double nx = 0.0, nt = 0.0;
     for (int j0 = 0; j0 < nseg; j0 += 32) {
-        double2 part = make_double2(0.0, 0.0);
-        if (j0 + lane < nseg) part = *reinterpret_cast<const double2*>(a.part_norm + ((j0 + lane) * a.M_pad + row) * 2);
+        if (j0 > 0) {
+            part = make_double2(0.0, 0.0);
+            if (j0 + lane < nseg)
+                part = *reinterpret_cast<const double2*>(a.part_norm + ((j0 + lane) * a.M_pad + row) * 2);
+        }
         const int m = nseg - j0 < 32 ? nseg - j0 : 32;
         for (int j = 0; j < m; ++j) {
             nx += __shfl_sync(0xFFFFFFFFu, part.x, j);
@@ -384,23 +408,29 @@ __global__ void __launch_bounds__(256) rtlynx_scale_kernel(const ScaleArgs a) {
         }
     }
     const float s = static_cast<float>(sqrt(nx) / (sqrt(nt) + 1e-8));
-    if (lane == 0) a.s_out[row] = s;
-    for (int i0 = lane;;) {
+    if (lane == 0) {
+        s_sh[w] = s;
+        a.s_out[row] = s;
+    }
+    __syncthreads();
+    for (int i0 = static_cast<int>(threadIdx.x);;) {
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-            if (i0 + 32 * u < n16) {
-                q[u].x = scale_pair(s, q[u].x);
-                q[u].y = scale_pair(s, q[u].y);
-                q[u].z = scale_pair(s, q[u].z);
-                q[u].w = scale_pair(s, q[u].w);
-                v[i0 + 32 * u] = q[u];
+            const int idx = i0 + 256 * u;
+            if (idx < total) {
+                const float sr = s_sh[idx / n16];
+                q[u].x = scale_pair(sr, q[u].x);
+                q[u].y = scale_pair(sr, q[u].y);
+                q[u].z = scale_pair(sr, q[u].z);
+                q[u].w = scale_pair(sr, q[u].w);
+                v[idx] = q[u];
             }
         }
-        i0 += 32 * kU;
-        if (i0 >= n16) break;
+        i0 += 256 * kU;
+        if (i0 >= total) break;
 #pragma unroll
         for (int u = 0; u < kU; ++u)
-            if (i0 + 32 * u < n16) q[u] = v[i0 + 32 * u];
+            if (i0 + 256 * u < total) q[u] = v[i0 + 256 * u];
     }
 }
 
