@@ -336,6 +336,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 // ---------------------------------------------------------------- pass 2
 struct ScaleArgs {
     int64_t M_pad, Kc_pad, total_tiles, grid;
+    int64_t trigger_from;  // CTAs from this index on (the last wave) let the GEMM launch
     int kt2, R_pad;
     const double* part_norm;
     const float* part_T;
@@ -361,7 +362,10 @@ __global__ void __launch_bounds__(256, 4) rtlynx_scale_kernel(const ScaleArgs a)
     const int64_t row = row0 + w;
     const int64_t first = (row0 / kBM) * a.kt2;
     grid_dependency_wait();  // everything pass 1 wrote is visible from here on
-    launch_dependents();
+    // Only the last wave lets the GEMM launch (the CTAs before it count once
+    // they exit): a GEMM CTA placed on an SM early would halve the room for
+    // the scale pass's later waves there.
+    if (static_cast<int64_t>(blockIdx.x) >= a.trigger_from) launch_dependents();
     const int64_t c0 = stream_owner_dev(first, a.total_tiles, a.grid);
     const int nseg = static_cast<int>(stream_owner_dev(first + a.kt2 - 1, a.total_tiles, a.grid) - c0 + 1);
     uint4* v = reinterpret_cast<uint4*>(a.vals + row0 * a.Kc_pad);
@@ -514,6 +518,10 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
 
     ScaleArgs b;
     b.M_pad = d.M_pad;
+    {
+        const int64_t ctas = d.M_pad / 8, wave = 4 * d.grid1;  // four scale CTAs fit on an SM
+        b.trigger_from = ctas > wave ? ctas - wave : 0;
+    }
     b.Kc_pad = d.Kc_pad;
     b.total_tiles = a.total_tiles;
     b.grid = d.grid1;
