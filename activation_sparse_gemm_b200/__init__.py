@@ -8,6 +8,7 @@ stream handle (int) or a ``torch.cuda.Stream``.
 
     Y = S(X) W^T + X (L_A L_B)^T        mode = MODE_SPARSE
     Y = X W^T                           mode = MODE_DENSE_SKIP
+    H = GELU(up(X)), Y = down(H)        rtlynx_mlp_block (two such layers)
 
 (RT-Lynx summary page, four-step pipeline paragraph, steps 1-3.)
 
@@ -36,7 +37,8 @@ ERR_DEVICE_TIMEOUT = 5
 ABI_SYMBOLS = (
     "rtlynx_linear", "rtlynx_workspace_size", "rtlynx_linear_ws", "rtlynx_linear_ws_events",
     "rtlynx_workspace_layout",
-    "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_linear_noalloc", "rtlynx_kernel_launches",
+    "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_mlp_block", "rtlynx_linear_noalloc",
+    "rtlynx_kernel_launches",
     "rtlynx_wait_selftest", "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
 )
 
@@ -81,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_sparsify_debug.restype = i
         L.rtlynx_linear_host.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i, p, p, p]
         L.rtlynx_linear_host.restype = i
+        L.rtlynx_mlp_block.argtypes = [p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i, i, p]
+        L.rtlynx_mlp_block.restype = i
         L.rtlynx_linear_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i, p, p]
         L.rtlynx_linear_noalloc.restype = i
         L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
@@ -124,6 +128,14 @@ def _check(status: int, what: str) -> int:
 def rtlynx_linear(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, stream=None) -> int:
     return _check(lib().rtlynx_linear(_ptr(X), _ptr(W), _ptr(L_A), _ptr(L_B), _ptr(Y), M, D_in, D_out, R,
                                       mode, _stream(stream)), "rtlynx_linear")
+
+
+def rtlynx_mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, H, Y, M, D, D_ff, R, mode_up=MODE_SPARSE,
+                     mode_down=MODE_SPARSE, stream=None) -> int:
+    """H = GELU(layer_up(X)) [M, D_ff], Y = layer_down(H) [M, D]; see include/rtlynx.h."""
+    return _check(lib().rtlynx_mlp_block(_ptr(X), _ptr(W_up), _ptr(LA_up), _ptr(LB_up), _ptr(W_down), _ptr(LA_down),
+                                         _ptr(LB_down), _ptr(H), _ptr(Y), M, D, D_ff, R, mode_up, mode_down,
+                                         _stream(stream)), "rtlynx_mlp_block")
 
 
 def rtlynx_workspace_size(M, D_in, D_out, R, mode) -> int:

@@ -272,6 +272,38 @@ static int cached_workspace(int dev, cudaStream_t stream, size_t bytes, void** o
     return RTLYNX_OK;
 }
 
+// One linear layer on a validated problem: the sparse path (prologue, then
+// the GEMM with LoRA) or the dense-skip GEMM; `act` selects the epilogue
+// activation.  Events (any may be null) are recorded before the first kernel,
+// between prologue and GEMM, and after the GEMM.
+static int run_layer(DeviceInfo* di, const void* X, const void* W, const void* L_A, const void* L_B, void* Y,
+                     int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, int act, void* workspace,
+                     size_t ws_bytes, void* ev_start, void* ev_mid, void* ev_end, cudaStream_t stream) {
+    const bool lora = (mode == RTLYNX_MODE_SPARSE) && R > 0 && L_A && L_B;
+    const Dims d = make_dims(M, D_in, D_out, lora ? R : 0, di->num_sms);
+    auto record = [&](void* ev) {
+        return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev), stream) == cudaSuccess;
+    };
+    if (mode == RTLYNX_MODE_DENSE_SKIP) {
+        Workspace none{};
+        if (!record(ev_start) || !record(ev_mid)) return RTLYNX_ERR_CUDA;
+        if (launch_gemm(d, false, X, W, nullptr, none, Y, act, di->num_sms, di->err_word, stream))
+            return RTLYNX_ERR_CUDA;
+        return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+    }
+    const WsLayout l = make_ws_layout(d);
+    if (!workspace || ws_bytes < l.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return RTLYNX_ERR_INVALID_ARG;
+    const Workspace ws = carve(workspace, l);
+    if (!record(ev_start)) return RTLYNX_ERR_CUDA;
+    int rc = run_prologue(d, X, lora ? L_B : nullptr, ws, di->err_word, di->num_sms, stream);
+    if (rc) return rc;
+    if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
+    if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, act, di->num_sms, di->err_word, stream))
+        return RTLYNX_ERR_CUDA;
+    return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+}
+
 // Which prologue runs: the one-pass cluster kernel (returns its cluster size)
 // or the two-pass path (returns 0).
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
@@ -321,29 +353,8 @@ int rtlynx_linear_ws_events(const void* X, const void* W, const void* L_A, const
     DeviceInfo* di = nullptr;
     rc = current_device(&di);
     if (rc) return rc;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    const bool lora = (mode == RTLYNX_MODE_SPARSE) && R > 0 && L_A && L_B;
-    const Dims d = make_dims(M, D_in, D_out, lora ? R : 0, di->num_sms);
-    auto record = [&](void* ev) {
-        return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev), stream) == cudaSuccess;
-    };
-    if (mode == RTLYNX_MODE_DENSE_SKIP) {
-        Workspace none{};
-        if (!record(ev_start) || !record(ev_mid)) return RTLYNX_ERR_CUDA;
-        if (launch_gemm(d, false, X, W, nullptr, none, Y, di->num_sms, di->err_word, stream)) return RTLYNX_ERR_CUDA;
-        return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
-    }
-    const WsLayout l = make_ws_layout(d);
-    if (!workspace || ws_bytes < l.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return RTLYNX_ERR_INVALID_ARG;
-    const Workspace ws = carve(workspace, l);
-    if (!record(ev_start)) return RTLYNX_ERR_CUDA;
-    rc = run_prologue(d, X, lora ? L_B : nullptr, ws, di->err_word, di->num_sms, stream);
-    if (rc) return rc;
-    if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
-    if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, di->num_sms, di->err_word, stream))
-        return RTLYNX_ERR_CUDA;
-    return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+    return run_layer(di, X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, 0, workspace, ws_bytes, ev_start, ev_mid, ev_end,
+                     static_cast<cudaStream_t>(stream_));
 }
 
 int rtlynx_linear_ws(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
@@ -370,6 +381,42 @@ int rtlynx_linear(const void* X, const void* W, const void* L_A, const void* L_B
     rc = cached_workspace(dev, static_cast<cudaStream_t>(stream_), bytes, &ws);
     if (rc) return rc;
     return rtlynx_linear_ws(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, ws, bytes, stream_);
+}
+
+int rtlynx_mlp_block(const void* X, const void* W_up, const void* LA_up, const void* LB_up, const void* W_down,
+                     const void* LA_down, const void* LB_down, void* H, void* Y, int64_t M, int64_t D, int64_t D_ff,
+                     int64_t R, int mode_up, int mode_down, void* stream_) {
+    int rc = validate(X, W_up, LA_up, LB_up, H, M, D, D_ff, R, mode_up);
+    if (rc) return rc;
+    rc = validate(H, W_down, LA_down, LB_down, Y, M, D_ff, D, R, mode_down);
+    if (rc) return rc;
+    if (H == X || H == Y || Y == X) return RTLYNX_ERR_INVALID_ARG;
+    DeviceInfo* di = nullptr;
+    rc = current_device(&di);
+    if (rc) return rc;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    auto ws_bytes = [&](int64_t K, int64_t N, const void* la, const void* lb, int mode) -> size_t {
+        if (mode == RTLYNX_MODE_DENSE_SKIP) return 0;
+        const bool lora = R > 0 && la && lb;
+        return make_ws_layout(make_dims(M, K, N, lora ? R : 0, di->num_sms)).total;
+    };
+    const size_t b_up = ws_bytes(D, D_ff, LA_up, LB_up, mode_up);
+    const size_t b_dn = ws_bytes(D_ff, D, LA_down, LB_down, mode_down);
+    const size_t bytes = b_up > b_dn ? b_up : b_dn;
+    void* ws = nullptr;
+    if (bytes > 0) {
+        rc = cached_workspace(dev, stream, bytes, &ws);
+        if (rc) return rc;
+    }
+    // up-projection with GELU in its epilogue, then the down-projection; the
+    // two layers use the workspace one after the other in stream order
+    rc = run_layer(di, X, W_up, LA_up, LB_up, H, M, D, D_ff, R, mode_up, 1, ws, bytes, nullptr, nullptr, nullptr,
+                   stream);
+    if (rc) return rc;
+    return run_layer(di, H, W_down, LA_down, LB_down, Y, M, D_ff, D, R, mode_down, 0, ws, bytes, nullptr, nullptr,
+                     nullptr, stream);
 }
 
 int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_in, int64_t R, void* vals,

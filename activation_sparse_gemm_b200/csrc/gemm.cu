@@ -22,8 +22,9 @@
 //               dense tcgen05.mma for the LoRA stages into the SAME accumulator,
 //               so T L_A^T never leaves the chip.  Its commits arrive on the
 //               barriers of both CTAs.
-//   warps 2-5   epilogue: tcgen05.ld, round to bf16, swizzled staging in shared
-//               memory, TMA store (clips the ragged M and N edges).
+//   warps 2-5   epilogue: tcgen05.ld, optional GELU, round to bf16, swizzled
+//               staging in shared memory, TMA store (clips the ragged M and N
+//               edges).
 // The accumulator is double-buffered in tensor memory, so the epilogue of one
 // tile overlaps the main loop of the next.
 //
@@ -90,6 +91,27 @@ struct PairArgs {
     uint16_t* Y;        // [M, N] bf16 output, row-major (the dense-skip epilogue stores to it directly)
     int* err;
 };
+
+// GELU, erf form: x * Phi(x) = x/2 (1 + erf(x / sqrt 2)), in float.
+// erfc(z) for z = |x| / sqrt 2 >= 0 comes from Hastings' rational
+// approximation as printed in Abramowitz & Stegun, Handbook of Mathematical
+// Functions, formula 7.1.26: erfc(z) ~ (a1 t + ... + a5 t^5) exp(-z^2) with
+// t = 1 / (1 + p z), absolute error at most 1.5e-7.  Working with erfc
+// avoids the cancellation of 1 + erf for negative x:
+//   x >= 0:  GELU = x (1 - erfc(z) / 2),    x < 0:  GELU = x erfc(z) / 2.
+// About fifteen instructions (one reciprocal, one exponential), so the GEMM
+// epilogue stays cheaper than the main loop it overlaps.
+__device__ __forceinline__ float gelu_erf(float x) {
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+    float poly = fmaf(t, 1.061405429f, -1.453152027f);
+    poly = fmaf(t, poly, 1.421413741f);
+    poly = fmaf(t, poly, -0.284496736f);
+    poly = fmaf(t, poly, 0.254829592f);
+    poly *= t;
+    const float half_erfc = 0.5f * poly * __expf(-z * z);
+    return x >= 0.0f ? fmaf(-x, half_erfc, x) : x * half_erfc;
+}
 
 // Raster order of the tiles: column tiles are taken in groups of group_n; a
 // group's tiles are numbered row pair by row pair, so a wave of consecutive
@@ -176,7 +198,7 @@ __device__ __forceinline__ void store_row_bf16(const PairArgs& a, int row, int c
     }
 }
 
-template <bool SPARSE, int BN>
+template <bool SPARSE, int BN, int ACT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     rtlynx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmLA,
@@ -505,6 +527,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                             }
                         }
                     }
+                    if constexpr (ACT == 1) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(gelu_erf(__uint_as_float(r[q])));
+                    }
                     if constexpr (!SPARSE) {
                         store_row_bf16(args, row0 + lane, col0 + c, half, r);
                         continue;
@@ -569,12 +595,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
 }
 
-template <bool SPARSE, int BN>
+template <bool SPARSE, int BN, int ACT>
 static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmT,
                        const CUtensorMap& tmLA, const CUtensorMap& tmE, const CUtensorMap& tmY,
                        const CUtensorMap& tmY16, const PairArgs& args, int num_sms, cudaStream_t stream) {
     using G = PairShape<SPARSE, BN>;
-    auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN>;
+    auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN, ACT>;
     static std::atomic<uint64_t> smem_set{0};
     const int e = allow_max_dynamic_smem(kernel, smem_set);
     if (e) return e;
@@ -589,7 +615,7 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
 }
 
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
-                void* Y, int num_sms, int* err, cudaStream_t stream) {
+                void* Y, int act, int num_sms, int* err, cudaStream_t stream) {
     constexpr int BN = kPairBN;
     CUtensorMap tmA, tmB, tmT, tmLA, tmE, tmY, tmY16;
     int rc;
@@ -664,8 +690,12 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.split_cnt = ws.split_cnt;
     args.Y = static_cast<uint16_t*>(Y);
     args.err = err;
-    return sparse ? launch_pair<true, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
-                  : launch_pair<false, BN>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
+    // the epilogue activation is a template parameter, so the plain kernels carry no GELU code
+    if (act == 1)
+        return sparse ? launch_pair<true, BN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
+                      : launch_pair<false, BN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
+    return sparse ? launch_pair<true, BN, 0>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
+                  : launch_pair<false, BN, 0>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
 }
 
 }  // namespace rtlynx

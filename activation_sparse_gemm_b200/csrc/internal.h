@@ -117,8 +117,9 @@ int allow_max_dynamic_smem(Kernel kernel, std::atomic<uint64_t>& done) {
 // The sparsify prologue: two launches (streaming pass, then per-token scale).
 int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err,
                     cudaStream_t stream);
+// act: 0 none, 1 GELU (erf form) applied to the output before its bf16 rounding.
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
-                void* Y, int num_sms, int* err, cudaStream_t stream);
+                void* Y, int act, int num_sms, int* err, cudaStream_t stream);
 // Shared by the entry points (api.cu).
 bool ensure_tmap_encoder();
 Workspace carve(void* base, const WsLayout& l);

@@ -99,7 +99,7 @@ extern "C" int rtlynx_linear_noalloc(const void* X, const void* W, const void* L
     const Dims d = make_dims(M, D_in, D_out, lora ? R : 0, nd->num_sms);
     if (mode == RTLYNX_MODE_DENSE_SKIP) {
         Workspace none{};
-        return launch_gemm(d, false, X, W, nullptr, none, Y, nd->num_sms, dev_status, stream) ? RTLYNX_ERR_CUDA
+        return launch_gemm(d, false, X, W, nullptr, none, Y, 0, nd->num_sms, dev_status, stream) ? RTLYNX_ERR_CUDA
                                                                                               : RTLYNX_OK;
     }
     const WsLayout l = make_ws_layout(d);
@@ -107,7 +107,7 @@ extern "C" int rtlynx_linear_noalloc(const void* X, const void* W, const void* L
     const Workspace ws = carve(nd->scratch, l);
     rc = run_prologue(d, X, lora ? L_B : nullptr, ws, dev_status, nd->num_sms, stream);
     if (rc) return rc;
-    if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, nd->num_sms, dev_status, stream))
+    if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, 0, nd->num_sms, dev_status, stream))
         return RTLYNX_ERR_CUDA;
     return RTLYNX_OK;
 }

@@ -109,3 +109,13 @@ def make_inputs(wl: Workload, M: int | None = None, weights: bool = True):
 def make_custom(M: int, K: int, N: int, R: int, seed: int, p_out: float = 0.08, gelu: bool = False):
     """Same recipe at an arbitrary shape (edge cases and ragged tails)."""
     return make_inputs(Workload("custom", M, K, N, R, p_out, seed, gelu))
+
+
+def make_block_inputs(M: int, D: int, D_ff: int, R: int, seed: int, p_out: float = 0.05):
+    """Inputs of a DiT feed-forward block (two layers): the up-projection's X,
+    W_up [D_ff, D], LA_up, LB_up with the recipe above (seed), and the
+    down-projection's W_down [D, D_ff], LA_down, LB_down drawn from seed + 100.
+    The down-projection's input is produced by the block itself."""
+    X, W_up, LA_up, LB_up = make_custom(M, D, D_ff, R, seed, p_out=p_out)
+    _, W_down, LA_down, LB_down = make_custom(1, D_ff, D, R, seed + 100, p_out=0.0)
+    return X, W_up, LA_up, LB_up, W_down, LA_down, LB_down

@@ -1,6 +1,7 @@
 """Benchmark of the RT-Lynx fused activation-sparse + LoRA linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qkv] [--impl ours|reference]
+    python bench.py --workload dit_mlp   (the feed-forward block of two layers, one GPU)
 
 One step = one call of the whole layer (sparsify prologue with the LoRA
 down-projection, then the sparse GEMM with the LoRA up-projection accumulated
@@ -358,6 +359,87 @@ def profiled_traffic(workload):
         return None
 
 
+def run_block(args):
+    """The DiT feed-forward block (rtlynx_mlp_block): up-projection with GELU in
+    its epilogue, then the down-projection, at the MLP workloads' shape; one
+    JSON line.  cuBLAS matmul + torch GELU + matmul on the same tensors is
+    timed in the same run."""
+    import numpy as np
+    import torch
+
+    import activation_sparse_gemm_b200 as rl
+    from activation_sparse_gemm_b200.inputs import make_block_inputs
+
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    rl.lib()
+    M, D, D_ff, R = 4608, 3072, 12288, 64
+    host = make_block_inputs(M, D, D_ff, R, seed=2)
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+    X, W_up, LA_up, LB_up, W_down, LA_down, LB_down = [dev(a) for a in host]
+    H = torch.empty((M, D_ff), dtype=torch.bfloat16, device=device)
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        pairs = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            a = ev()
+            fn()
+            b = ev()
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in pairs)
+
+    def block(mu, md):
+        return lambda: rl.rtlynx_mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, H, Y, M, D, D_ff, R,
+                                           mu, md, stream)
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    ms = timed(block(rl.MODE_SPARSE, rl.MODE_SPARSE))
+    clocks.stop()
+    status = rl.rtlynx_stream_status(stream)
+    if status != rl.OK:
+        raise RuntimeError(f"device-side error: {rl.rtlynx_status_string(status)}")
+    skip_down_ms = timed(block(rl.MODE_SPARSE, rl.MODE_DENSE_SKIP))
+    gelu = torch.nn.GELU()
+
+    def cublas_chain():
+        torch.matmul(gelu(torch.matmul(X, W_up.t())), W_down.t(), out=Y)
+
+    cublas_ms = timed(cublas_chain)
+    flop = 2 * 2 * M * D * D_ff + 2 * 2 * M * R * (D + D_ff)
+    launches = (rl.rtlynx_kernel_launches(M, D, D_ff, R, rl.MODE_SPARSE) +
+                rl.rtlynx_kernel_launches(M, D_ff, D, R, rl.MODE_SPARSE))
+    line = {
+        "metric": "DiT feed-forward block (up + GELU + down, both RT-Lynx sparse): us/call, TFLOP/s, "
+                  "speedup vs cuBLAS dense chain",
+        "value": flop / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
+        "dense_chain_cublas_us": cublas_ms * 1e3, "speedup_vs_dense_chain": cublas_ms / ms,
+        "down_skipped_us": skip_down_ms * 1e3, "dtype": "bf16", "vs_baseline": None,
+        "data": "synthetic (seeded, DiT-shaped; random-init weights)",
+        "config": {"workload": f"dit_mlp: M={M} D={D} D_ff={D_ff} R={R}", "M": M, "D": D, "D_ff": D_ff, "R": R,
+                   "l2": "flushed before every timed step (256 MB write)"},
+        "gpu_launches": launches * args.steps, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def kernel_rev():
     """Hash of the GEMM kernel source, to tell whether stored ncu counters still apply."""
     import hashlib
@@ -368,6 +450,8 @@ def kernel_rev():
 def main():
     args = parse()
     from activation_sparse_gemm_b200.inputs import WORKLOADS
+    if args.workload == "dit_mlp" and args.impl == "ours":
+        return run_block(args)
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)

@@ -117,6 +117,30 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
                        int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* X_dev, void* Y_dev,
                        void* stream);
 
+/*
+ * rtlynx_mlp_block - the feed-forward part of a DiT block built from two
+ * RT-Lynx linear layers (RT-Lynx summary page, four-step pipeline paragraph:
+ * steps 1-2 for each layer, step 3 for layers chosen for skipping):
+ *   H = GELU(layer_up(X))      [M, D_ff], GELU in its erf form,
+ *                              x/2 (1 + erf(x/sqrt 2)), applied in the
+ *                              up-projection's epilogue before the bf16
+ *                              rounding of H (no separate pass)
+ *   Y = layer_down(H)          [M, D]
+ * Each layer runs as rtlynx_linear with its own mode (mode_up, mode_down:
+ * RTLYNX_MODE_SPARSE or RTLYNX_MODE_DENSE_SKIP, selective layer skipping)
+ * and LoRA pair; both pairs have rank R.
+ *   X [M, D], W_up [D_ff, D], LA_up [D_ff, R], LB_up [R, D],
+ *   W_down [D, D_ff], LA_down [D, R], LB_down [R, D_ff], all bf16, device.
+ *   H  caller-owned [M, D_ff] bf16 device buffer that receives the GELU
+ *      activations (the down-projection's input); it must not overlap X or Y.
+ *   D and D_ff multiples of 8.
+ * Uses the workspace cache of rtlynx_linear (sized for the larger layer).
+ * Argument errors of either layer return before anything is launched.
+ */
+int rtlynx_mlp_block(const void* X, const void* W_up, const void* LA_up, const void* LB_up, const void* W_down,
+                     const void* LA_down, const void* LB_down, void* H, void* Y, int64_t M, int64_t D, int64_t D_ff,
+                     int64_t R, int mode_up, int mode_down, void* stream);
+
 /* Largest workspace rtlynx_linear_noalloc can use (32 MiB). */
 #define RTLYNX_NOALLOC_MAX_BYTES (32u << 20)
 

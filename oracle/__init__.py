@@ -7,7 +7,8 @@ The arithmetic lives in ``rtlynx_oracle.c`` (plain C, double precision, plain
 triple-loop GEMMs, OpenMP over tokens).  It follows the four-step pipeline
 paragraph of the RT-Lynx summary page (paper.rainbus.top, arXiv 2605.26632),
 steps 1-3: Top-K 2-of-4 mask, norm-compensating scale s, LoRA branch on the
-dense X, and the dense path for skipped layers.  This module only compiles the
+dense X, and the dense path for skipped layers; plus the feed-forward block of
+two such layers joined by GELU (erf form).  This module only compiles the
 C file with gcc and marshals numpy arrays through ctypes.
 """
 from __future__ import annotations
@@ -63,6 +64,10 @@ class Oracle:
         lib.oracle_linear_rows.restype = ctypes.c_int
         lib.oracle_bf16_from_double.argtypes = [ctypes.c_double]
         lib.oracle_bf16_from_double.restype = ctypes.c_uint16
+        lib.oracle_gelu_bf16.argtypes = [p, i64, p]
+        lib.oracle_gelu_bf16.restype = ctypes.c_int
+        lib.oracle_gelu.argtypes = [ctypes.c_double]
+        lib.oracle_gelu.restype = ctypes.c_double
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         self.lib = lib
@@ -120,6 +125,28 @@ class Oracle:
         return Y
 
 
+    def gelu(self, y: float) -> float:
+        """GELU (erf form) of one double, in double."""
+        return float(self.lib.oracle_gelu(float(y)))
+
+    def gelu_bf16(self, Y: np.ndarray) -> np.ndarray:
+        """bf16 bits of GELU(Y) (erf form, double, one rounding), same shape as Y."""
+        Y = np.ascontiguousarray(Y, dtype=np.float64)
+        H = np.empty(Y.shape, np.uint16)
+        if self.lib.oracle_gelu_bf16(_ptr(Y), Y.size, _ptr(H)):
+            raise ValueError("oracle_gelu_bf16 rejected its arguments")
+        return H
+
+    def mlp_block(self, X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up: int = MODE_SPARSE,
+                  mode_down: int = MODE_SPARSE, rows=None):
+        """The DiT feed-forward block of two layers: H = bf16(GELU(layer_up(X))) and
+        Y = layer_down(H), for the listed tokens (all when rows is None; tokens are
+        independent).  Returns (Y_up float64, H bf16 bits, Y float64)."""
+        Y_up = self.linear(X, W_up, LA_up, LB_up, mode=mode_up, rows=rows)
+        H = self.gelu_bf16(Y_up)
+        Y = self.linear(H, W_down, LA_down, LB_down, mode=mode_down)
+        return Y_up, H, Y
+
 def _default() -> Oracle:
     global _lib
     if _lib is None:
@@ -141,3 +168,17 @@ def sparsify(X):
 
 def linear(X, W, L_A=None, L_B=None, mode: int = MODE_SPARSE, rows=None, want_T: bool = False):
     return _default().linear(X, W, L_A, L_B, mode=mode, rows=rows, want_T=want_T)
+
+
+def gelu(y: float) -> float:
+    return _default().gelu(y)
+
+
+def gelu_bf16(Y):
+    return _default().gelu_bf16(Y)
+
+
+def mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up: int = MODE_SPARSE,
+              mode_down: int = MODE_SPARSE, rows=None):
+    return _default().mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up=mode_up,
+                                mode_down=mode_down, rows=rows)

@@ -15,6 +15,8 @@
  *   S(X) = s * X~
  *   Y_s  = S(X) W^T,   Y_r = X (L_A L_B)^T  (dense X, rank R),   Y = Y_s + Y_r
  *   dense-skip layers ("Selective Layer Skipping", step 3): Y = X W^T
+ *   feed-forward block of two such layers: H = bf16(GELU(Y_up)), GELU in its
+ *   erf form, then Y = layer_down(H)
  *
  * Readings where the page is silent (each is listed in the design notes):
  *   - Top-K ranks by magnitude |x|; equal magnitudes go to the lower index;
@@ -76,11 +78,13 @@ double oracle_double_from_bf16(uint16_t b) { return bf16_to_double(b); }
 
 /* Top-K (2 of 4) on one group: index i is kept iff fewer than two other
  * entries beat it, where j beats i when |x_j| > |x_i|, or |x_j| == |x_i|
- * and j < i.  Returns the kept indices in ascending order. */
+ * and j < i.  Returns the kept indices in ascending order.  For finite
+ * entries exactly two are kept; a NaN (out of contract) compares false and
+ * could pass the test for more, so at most the first two are taken. */
 static void keep_two_of_four(const double x[4], int *i0, int *i1)
 {
-    int kept[2], n = 0;
-    for (int i = 0; i < 4; ++i) {
+    int kept[2] = {0, 1}, n = 0;
+    for (int i = 0; i < 4 && n < 2; ++i) {
         int beaten = 0;
         for (int j = 0; j < 4; ++j) {
             if (j == i) continue;
@@ -203,6 +207,22 @@ int oracle_linear_rows(const uint16_t *X, const uint16_t *W, const uint16_t *L_A
         free(Trow);
     }
     return bad ? 1 : 0;
+}
+
+/* The activation between the two layers of a DiT feed-forward block:
+ * GELU in its erf form, gelu(y) = y * Phi(y) = y/2 * (1 + erf(y / sqrt 2)),
+ * written as y/2 * erfc(-y / sqrt 2), the same function without the
+ * cancellation of 1 + erf for negative y.  Evaluated in double on the exact
+ * output of the first layer and rounded once to bf16 (nearest even): the
+ * block's intermediate activation is a bf16 tensor like every activation the
+ * layers exchange.  H [n] bf16 bits. */
+double oracle_gelu(double y) { return 0.5 * y * erfc(-y / sqrt(2.0)); }
+
+int oracle_gelu_bf16(const double *Y, int64_t n, uint16_t *H)
+{
+    if (n < 0) return 1;
+    for (int64_t i = 0; i < n; ++i) H[i] = double_to_bf16_rne(oracle_gelu(Y[i]));
+    return 0;
 }
 
 /* Threads the OpenMP runtime will use (reported next to CPU timings). */

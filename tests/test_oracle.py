@@ -332,3 +332,71 @@ def test_tiny_digest_unchanged():
     want = json.load(open(os.path.join(GOLDEN, "tiny_oracle.json")))
     got = mg.digest()
     assert got == want
+
+
+
+# ------------------------------------------------------------------ feed-forward block (GELU between two layers)
+def test_gelu_closed_forms():
+    """GELU(x) = x Phi(x): Phi(1) and Phi(2) from the standard normal table,
+    the identity GELU(x) - GELU(-x) = x, GELU(0) = 0, and the scipy routine."""
+    from scipy.special import ndtr
+    assert abs(oracle.gelu(1.0) - 0.8413447460685429) < 1e-15       # Phi(1)
+    assert abs(oracle.gelu(2.0) - 2 * 0.9772498680518208) < 1e-15   # 2 Phi(2)
+    assert oracle.gelu(0.0) == 0.0
+    rng = np.random.default_rng(7)
+    for x in rng.normal(0, 3, 200):
+        assert abs(oracle.gelu(x) - oracle.gelu(-x) - x) <= 1e-14 * max(1.0, abs(x))
+        assert abs(oracle.gelu(x) - x * ndtr(x)) <= 1e-14 * max(1.0, abs(x))
+    assert abs(oracle.gelu(10.0) - 10.0) < 1e-20 and abs(oracle.gelu(-10.0)) < 1e-20
+
+
+def test_gelu_bf16_is_one_rounding_of_the_exact_value():
+    """H = bf16(GELU(y)) rounded once, nearest even: compared with the exact
+    nearest bf16 of a 40-digit GELU value (skip values within 1e-12 relative of
+    a rounding boundary, where the double evaluation may land either side)."""
+    from scipy.special import ndtr
+    rng = np.random.default_rng(8)
+    y = np.concatenate([rng.normal(0, 2, 3000), rng.normal(0, 40, 1000), [0.0, -0.0, 1e-30, -5.5, 3.25]])
+    H = oracle.gelu_bf16(y)
+    checked = 0
+    for yi, hb in zip(y, H):
+        g = Fraction(float(yi)) * Fraction(float(ndtr(yi)))
+        lo = nearest_bf16_bits(g * (1 - Fraction(1, 10 ** 12)))
+        hi = nearest_bf16_bits(g * (1 + Fraction(1, 10 ** 12)))
+        if lo == hi:
+            def z(b):  # +0 and -0 are the same value (GELU of a large negative y rounds to a zero)
+                return 0 if b == 0x8000 else b
+            assert z(int(hb)) == z(lo), (yi, hex(int(hb)), hex(lo))
+            checked += 1
+    assert checked > 3900
+
+
+def test_mlp_block_wiring_with_selection_weights():
+    """Up-projection dense-skip with W_up selecting input channels (rows of the
+    identity): Y_up = X exactly, so H = bf16(GELU(X)).  Down-projection
+    dense-skip with W_down = identity: Y = H.  Tokens are independent, so a row
+    subset equals the same rows of the whole."""
+    M, D = 24, 32
+    X, _, _, _ = make_custom(M, D, 8, 8, seed=41)
+    eye = to_bf16_bits(np.eye(D, dtype=np.float32))
+    Y_up, H, Y = oracle.mlp_block(X, eye, None, None, eye, None, None,
+                                  mode_up=oracle.MODE_DENSE_SKIP, mode_down=oracle.MODE_DENSE_SKIP)
+    xf = f64(X)
+    assert (Y_up == xf).all()
+    assert (H == oracle.gelu_bf16(xf)).all()
+    assert (Y == f64(H)).all()
+    rows = [3, 0, 17]
+    Y_up2, H2, Y2 = oracle.mlp_block(X, eye, None, None, eye, None, None,
+                                     mode_up=oracle.MODE_DENSE_SKIP, mode_down=oracle.MODE_DENSE_SKIP, rows=rows)
+    assert (Y_up2 == Y_up[rows]).all() and (H2 == H[rows]).all() and (Y2 == Y[rows]).all()
+
+
+def test_mlp_block_sparse_rows_subset():
+    from activation_sparse_gemm_b200.inputs import make_block_inputs
+    args = make_block_inputs(40, 64, 128, 16, seed=9)
+    _, H, Y = oracle.mlp_block(*args)
+    rows = [39, 2, 11]
+    _, H2, Y2 = oracle.mlp_block(*args, rows=rows)
+    assert (H2 == H[rows]).all() and (Y2 == Y[rows]).all()
+    # GELU output is never below its minimum, about -0.17
+    assert (bf16_bits_to_f32(H) >= -0.1701).all()
