@@ -264,8 +264,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const uint32_t tmem_meta = tmem_base + 2 * BN;
-    // In sparse mode the GEMM is launched as a programmatic dependent of the
-    // prologue: the setup above overlaps its tail, the operands are read after this.
+    // The GEMM is launched as a programmatic dependent of the preceding kernel
+    // (the prologue in sparse mode): the setup above overlaps its tail, the
+    // operands are read after this.
     grid_dependency_wait();
 
     PairWork w;
@@ -607,11 +608,11 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
     const int tiles = args.m_pairs * args.n_tiles;
     const int max_pairs = num_sms / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
-    if (SPARSE)  // follows the scale pass of the prologue
-        return launch_dependent(kernel, dim3(2 * pairs), dim3(kPairThreads), G::SMEM_BYTES, stream, tmA, tmB, tmT,
-                                tmLA, tmE, tmY, tmY16, args);
-    kernel<<<2 * pairs, kPairThreads, G::SMEM_BYTES, stream>>>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args);
-    return cudaGetLastError();
+    // A programmatic dependent of whatever ran before (the prologue in sparse
+    // mode): the setup overlaps that kernel's tail, the operands are read
+    // after grid_dependency_wait.
+    return launch_dependent(kernel, dim3(2 * pairs), dim3(kPairThreads), G::SMEM_BYTES, stream, tmA, tmB, tmT, tmLA,
+                            tmE, tmY, tmY16, args);
 }
 
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,

@@ -118,6 +118,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = LORA ? *tmem_holder : 0u;
+    // Launched as a programmatic dependent: the setup above overlaps the tail
+    // of whatever ran before in the stream (the previous layer's GEMM, say),
+    // and nothing before this wait touches memory that kernel may still use.
+    grid_dependency_wait();
     launch_dependents();  // the scale pass may be scheduled; it waits for this grid to finish
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.n_split_cnt; i += blockDim.x) a.split_cnt[i] = 0;
@@ -504,16 +508,10 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
     const dim3 grid(static_cast<unsigned>(d.grid1));
     cudaError_t e;
     static std::atomic<uint64_t> smem_set[2];
-    if (lora) {
-        const int rc2 = allow_max_dynamic_smem(rtlynx_sparsify_stream_kernel<true>, smem_set[1]);
-        if (rc2) return rc2;
-        rtlynx_sparsify_stream_kernel<true><<<grid, kStreamThreads, smem, stream>>>(tmX, tmLB, a);
-    } else {
-        const int rc2 = allow_max_dynamic_smem(rtlynx_sparsify_stream_kernel<false>, smem_set[0]);
-        if (rc2) return rc2;
-        rtlynx_sparsify_stream_kernel<false><<<grid, kStreamThreads, smem, stream>>>(tmX, tmLB, a);
-    }
-    e = cudaGetLastError();
+    auto kernel = lora ? rtlynx_sparsify_stream_kernel<true> : rtlynx_sparsify_stream_kernel<false>;
+    const int rc2 = allow_max_dynamic_smem(kernel, smem_set[lora ? 1 : 0]);
+    if (rc2) return rc2;
+    e = static_cast<cudaError_t>(launch_dependent(kernel, grid, dim3(kStreamThreads), smem, stream, tmX, tmLB, a));
     if (e != cudaSuccess) return e;
 
     ScaleArgs b;
