@@ -69,7 +69,8 @@ struct PairShape {
     static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-    static_assert(BN % 16 == 0 && BN >= 64 && 2 * BN + 4 <= 512, "two accumulators and the metadata must fit");
+    static_assert(BN % 16 == 0 && BN >= 64 && 2 * BN + (SPARSE ? 4 : 0) <= 512,
+                  "two accumulators (and, when sparse, the metadata) must fit");
     static_assert(B_ATOM_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
     static_assert(LORA_A_BYTES <= A_BYTES && LORA_B_BYTES <= B_BYTES, "LoRA tiles must fit the operand slots");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -617,7 +618,10 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
 
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
                 void* Y, int act, int num_sms, int* err, cudaStream_t stream) {
-    constexpr int BN = kPairBN;
+    // Sparse tiles are 240 wide so that two accumulators and the metadata fit
+    // in 512 tensor-memory columns; dense-skip tiles carry no metadata and are
+    // 256 wide (two accumulators fill the 512 columns).
+    const int BN = sparse ? kPairBN : kDenseBN;
     CUtensorMap tmA, tmB, tmT, tmLA, tmE, tmY, tmY16;
     int rc;
     if (sparse) {
@@ -693,10 +697,10 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.err = err;
     // the epilogue activation is a template parameter, so the plain kernels carry no GELU code
     if (act == 1)
-        return sparse ? launch_pair<true, BN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
-                      : launch_pair<false, BN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
-    return sparse ? launch_pair<true, BN, 0>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
-                  : launch_pair<false, BN, 0>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
+        return sparse ? launch_pair<true, kPairBN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
+                      : launch_pair<false, kDenseBN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
+    return sparse ? launch_pair<true, kPairBN, 0>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)
+                  : launch_pair<false, kDenseBN, 0>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
 }
 
 }  // namespace rtlynx

@@ -17,7 +17,8 @@ constexpr int kBN = 256;          // output columns per tile
 constexpr int kBK = 64;           // logical K per pipeline stage
 constexpr int kChunkK = 128;      // logical K per metadata chunk (4 sparse MMAs of K = 32)
 constexpr int kChunkBytes = 2048; // 128 lanes x 16 bytes of metadata per chunk
-constexpr int kPairBN = 240;      // output columns per GEMM tile (one CTA pair)
+constexpr int kPairBN = 240;      // output columns per sparse GEMM tile (one CTA pair)
+constexpr int kDenseBN = 256;     // output columns per dense-skip GEMM tile
 // fp32 partial of one CTA's 128 x 240 tile: [32-column chunk 8][4-column group 8][row 128][4]
 constexpr int kSplitSlotFloats = 8 * kBM * 32;
 constexpr int kMaxSplit = 6;  // parts of one split tile (the fix-up holds two chunks of the others in shared memory)
