@@ -75,6 +75,36 @@ int current_device(DeviceInfo** out) {
     return RTLYNX_OK;
 }
 
+// The host-buffer entry point pipelines its copies over token chunks on two
+// helper streams per device (uploads, downloads), created on first use.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join_up = nullptr, ev_join_down = nullptr;
+    cudaEvent_t ev_h2d[kHostChunks] = {}, ev_comp[kHostChunks] = {};
+};
+std::mutex g_host_mutex;
+HostPipe g_host[kMaxDevices];
+
+int host_pipe(int dev, HostPipe** out) {
+    HostPipe& hp = g_host[dev];
+    if (!hp.ready) {
+        auto ev = [](cudaEvent_t* e) { return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess; };
+        bool ok = cudaStreamCreateWithFlags(&hp.up, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&hp.down, cudaStreamNonBlocking) == cudaSuccess && ev(&hp.ev_fork) &&
+                  ev(&hp.ev_join_up) && ev(&hp.ev_join_down);
+        for (int i = 0; ok && i < kHostChunks; ++i) ok = ev(&hp.ev_h2d[i]) && ev(&hp.ev_comp[i]);
+        if (!ok) {
+            cudaGetLastError();
+            return RTLYNX_ERR_CUDA;
+        }
+        hp.ready = true;
+    }
+    *out = &hp;
+    return RTLYNX_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -448,16 +478,62 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
     if (!X_host || !Y_host) return RTLYNX_ERR_INVALID_ARG;
     int rc = validate(X_dev, W, L_A, L_B, Y_dev, M, D_in, D_out, R, mode);
     if (rc) return rc;
+    if (X_dev == Y_dev) return RTLYNX_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RTLYNX_ERR_CUDA;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    if (cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(M) * D_in * 2, cudaMemcpyHostToDevice, stream) !=
-        cudaSuccess)
-        return RTLYNX_ERR_CUDA;
-    rc = rtlynx_linear(X_dev, W, L_A, L_B, Y_dev, M, D_in, D_out, R, mode, stream_);
+    // At most kHostChunks token chunks of at least 512 rows; every chunk but
+    // the last is a whole number of 256-row blocks, so all of them fit the
+    // workspace the first one sizes.
+    int64_t n = M / 512;
+    n = n < 1 ? 1 : (n > kHostChunks ? kHostChunks : n);
+    const int64_t chunk = ((M + n - 1) / n + 255) / 256 * 256;
+    n = (M + chunk - 1) / chunk;
+    std::lock_guard<std::mutex> lock(g_host_mutex);  // the helper streams and events are shared per device
+    HostPipe* hp = nullptr;
+    rc = host_pipe(dev, &hp);
     if (rc) return rc;
-    if (cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(M) * D_out * 2, cudaMemcpyDeviceToHost, stream) !=
-        cudaSuccess)
+    if (cudaEventRecord(hp->ev_fork, stream) != cudaSuccess || cudaStreamWaitEvent(hp->up, hp->ev_fork, 0) != cudaSuccess)
         return RTLYNX_ERR_CUDA;
-    return RTLYNX_OK;
+    auto first = [&](int64_t i) { return i * chunk; };
+    auto rows = [&](int64_t i) { return (i + 1 < n ? chunk : M - i * chunk); };
+    const uint8_t* xh = static_cast<const uint8_t*>(X_host);
+    uint8_t* yh = static_cast<uint8_t*>(Y_host);
+    uint8_t* xd = static_cast<uint8_t*>(X_dev);
+    uint8_t* yd = static_cast<uint8_t*>(Y_dev);
+    const size_t xrow = static_cast<size_t>(D_in) * 2, yrow = static_cast<size_t>(D_out) * 2;
+    for (int64_t i = 0; i < n && rc == RTLYNX_OK; ++i) {
+        const size_t off = static_cast<size_t>(first(i)) * xrow, bytes = static_cast<size_t>(rows(i)) * xrow;
+        if (cudaMemcpyAsync(xd + off, xh + off, bytes, cudaMemcpyHostToDevice, hp->up) != cudaSuccess ||
+            cudaEventRecord(hp->ev_h2d[i], hp->up) != cudaSuccess)
+            rc = RTLYNX_ERR_CUDA;
+    }
+    int64_t issued = 0;  // chunks whose compute is queued
+    for (int64_t i = 0; i < n && rc == RTLYNX_OK; ++i) {
+        if (cudaStreamWaitEvent(stream, hp->ev_h2d[i], 0) != cudaSuccess) {
+            rc = RTLYNX_ERR_CUDA;
+            break;
+        }
+        rc = rtlynx_linear(xd + static_cast<size_t>(first(i)) * xrow, W, L_A, L_B,
+                           yd + static_cast<size_t>(first(i)) * yrow, rows(i), D_in, D_out, R, mode, stream_);
+        if (rc) break;
+        if (cudaEventRecord(hp->ev_comp[i], stream) != cudaSuccess ||
+            cudaStreamWaitEvent(hp->down, hp->ev_comp[i], 0) != cudaSuccess ||
+            cudaMemcpyAsync(yh + static_cast<size_t>(first(i)) * yrow, yd + static_cast<size_t>(first(i)) * yrow,
+                            static_cast<size_t>(rows(i)) * yrow, cudaMemcpyDeviceToHost, hp->down) != cudaSuccess) {
+            rc = RTLYNX_ERR_CUDA;
+            break;
+        }
+        ++issued;
+    }
+    // join: whatever was queued on the helper streams finishes before later work on `stream`
+    if (cudaEventRecord(hp->ev_join_up, hp->up) != cudaSuccess ||
+        cudaEventRecord(hp->ev_join_down, hp->down) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, hp->ev_join_up, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, hp->ev_join_down, 0) != cudaSuccess)
+        return RTLYNX_ERR_CUDA;
+    (void)issued;
+    return rc;
 }
 
 int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode) {
@@ -514,6 +590,26 @@ void rtlynx_release(void) {
         }
     }
     g_ws.clear();
+    {
+        std::lock_guard<std::mutex> hl(g_host_mutex);
+        for (int i = 0; i < kMaxDevices; ++i) {
+            HostPipe& hp = g_host[i];
+            if (!hp.ready) continue;
+            cudaSetDevice(i);
+            cudaStreamSynchronize(hp.up);
+            cudaStreamSynchronize(hp.down);
+            cudaStreamDestroy(hp.up);
+            cudaStreamDestroy(hp.down);
+            cudaEventDestroy(hp.ev_fork);
+            cudaEventDestroy(hp.ev_join_up);
+            cudaEventDestroy(hp.ev_join_down);
+            for (int c = 0; c < kHostChunks; ++c) {
+                cudaEventDestroy(hp.ev_h2d[c]);
+                cudaEventDestroy(hp.ev_comp[c]);
+            }
+            hp = HostPipe{};
+        }
+    }
     for (int i = 0; i < kMaxDevices; ++i) {
         if (g_dev[i].err_word) {
             cudaSetDevice(i);

@@ -110,9 +110,19 @@ int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_i
                           void* meta, void* s, void* T, void* stream);
 
 /* End-to-end form for callers whose activations live in host memory:
- * copies X_host (pinned for overlap) to X_dev, runs rtlynx_linear into Y_dev,
- * copies Y_dev to Y_host.  All three steps are queued on stream; synchronize
- * the stream before reading Y_host.  W, L_A, L_B are device pointers. */
+ * copies X_host to X_dev, runs rtlynx_linear into Y_dev, copies Y_dev to
+ * Y_host.  The work is cut into up to eight token chunks (of at least 512
+ * tokens) and pipelined: uploads run on one helper stream, each chunk's layer
+ * on `stream` once its upload has landed, downloads on a second helper stream
+ * once its layer is done, so copies in both directions overlap the compute.
+ * The helper streams belong to the library (one pair per device, created on
+ * the first call; make it outside any stream capture).  Everything is ordered
+ * after the work already queued on `stream`, and later work queued on
+ * `stream` waits for all of it; synchronize `stream` before reading Y_host.
+ * X_host and Y_host should be pinned (page-locked) for the copies to overlap.
+ * W, L_A, L_B, X_dev and Y_dev are device pointers; X_dev and Y_dev must not
+ * overlap.  Concurrent calls from several host threads are serialized while
+ * they enqueue. */
 int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const void* L_B, void* Y_host,
                        int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode, void* X_dev, void* Y_dev,
                        void* stream);

@@ -274,6 +274,36 @@ def test_full_workload_sampled(name):
         assert_y_close(Yd[rows], oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP, rows=rows), "mlp_down dense")
 
 
+# ------------------------------------------------------------------ host buffers in and out
+@pytest.mark.parametrize("M,K,N,R,mode", [(100, 256, 264, 16, rl.MODE_SPARSE), (3000, 256, 264, 16, rl.MODE_SPARSE),
+                                          (5000, 136, 136, 8, rl.MODE_SPARSE), (5000, 136, 136, 8, rl.MODE_DENSE_SKIP)])
+def test_linear_host_buffers_pipelined(M, K, N, R, mode):
+    """rtlynx_linear_host over 1, 4 and 7 token chunks (uploads, per-chunk
+    layers and downloads on three streams): Y in the pinned host buffer meets
+    the bar against the oracle, and later work on the caller's stream sees the
+    whole result."""
+    import torch
+    X, W, L_A, L_B = make_custom(M, K, N, R, seed=900 + M)
+    Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.full((M, N), float("nan"), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    Yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    lora = mode == rl.MODE_SPARSE
+    Wd = dev(W)
+    Ad, Bd = (dev(L_A), dev(L_B)) if lora else (None, None)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        rl.rtlynx_linear_host(Xh, Wd, Ad, Bd, Yh, M, K, N, R if lora else 0, mode, Xd, Yd, s)
+        Ycopy = Yd.clone()  # queued after the call on the same stream: must see every chunk
+    assert rl.rtlynx_stream_status(s) == rl.OK
+    s.synchronize()
+    Y = Yh.view(torch.int16).numpy().view(np.uint16)
+    ref = oracle.linear(X, W, L_A if lora else None, L_B if lora else None, mode=mode)
+    assert_y_close(Y, ref, f"host {M}x{K}x{N}", edge=True)
+    assert (host_bits(Ycopy) == Y).all()
+    assert (host_bits(Xd) == X).all()
+
+
 # ------------------------------------------------------------------ failure detection
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A device wait on a barrier nobody arrives on gives up, reports
