@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qkv] [--impl ours|reference]
     python bench.py --workload dit_mlp   (the feed-forward block of two layers, one GPU)
+    python bench.py --workload lora_fit  (the closed-form LoRA fit and the error it removes, one GPU)
 
 One step = one call of the whole layer (sparsify prologue with the LoRA
 down-projection, then the sparse GEMM with the LoRA up-projection accumulated
@@ -440,6 +441,63 @@ def run_block(args):
     return 0
 
 
+def run_lora_fit(args):
+    """The closed-form LoRA fit at the qkv shape: 4096 calibration tokens of the
+    qkv workload, R = 64; seconds per fit (CUDA events) and the relative error
+    of the sparse layer against the dense layer (both through the library) on
+    the calibration tokens and on 1024 further tokens of the same recipe."""
+    import numpy as np
+    import torch
+
+    import activation_sparse_gemm_b200 as rl
+    from activation_sparse_gemm_b200.inputs import WORKLOADS, make_inputs
+    from activation_sparse_gemm_b200.lora_fit import fit_lora
+
+    torch.cuda.set_device(0)
+    wl = WORKLOADS["qkv"]
+    M_cal, M_test = wl.M, 1024
+    X, W, L_A, L_B = make_inputs(wl, M=M_cal + M_test)
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    Xd, Wd, Ad, Bd = dev(X), dev(W), dev(L_A), dev(L_B)
+    K, N, R = wl.D_in, wl.D_out, wl.R
+    Xc, Xt = Xd[:M_cal].contiguous(), Xd[M_cal:].contiguous()
+    fit_lora(Xc, Wd, R)  # warm-up (library handles, workspaces)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    FA, FB = fit_lora(Xc, Wd, R)
+    b.record()
+    torch.cuda.synchronize()
+    fit_s = a.elapsed_time(b) / 1e3
+
+    def rel(Xs, LA, LB):
+        M = Xs.shape[0]
+        Yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        Ys = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        rl.rtlynx_linear(Xs, Wd, None, None, Yd, M, K, N, 0, rl.MODE_DENSE_SKIP)
+        rl.rtlynx_linear(Xs, Wd, LA, LB, Ys, M, K, N, R if LA is not None else 0, rl.MODE_SPARSE)
+        torch.cuda.synchronize()
+        d = Yd.double()
+        return float((Ys.double() - d).norm() / d.norm())
+
+    errs = {name: {"no_lora": rel(Xs, None, None), "random_lora": rel(Xs, Ad, Bd), "fitted_lora": rel(Xs, FA, FB)}
+            for name, Xs in (("calibration", Xc), ("held_out", Xt))}
+    line = {
+        "metric": "closed-form LoRA fit (reduced-rank regression on the sparsification residual): "
+                  "seconds per fit; relative error of the sparse layer against the dense layer",
+        "value": fit_s, "unit": "s", "higher_is_better": False, "n_gpus": 1, "steps": 1, "warmup": 1,
+        "rel_err_vs_dense": errs, "dtype": "bf16 layer, f64 fit", "vs_baseline": None,
+        "data": "synthetic (seeded qkv recipe: independent tokens, lognormal channel scales, outlier channels)",
+        "config": {"workload": f"lora_fit: calibration M={M_cal} held-out M={M_test} D_in={K} D_out={N} R={R}"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def kernel_rev():
     """Hash of the GEMM kernel source, to tell whether stored ncu counters still apply."""
     import hashlib
@@ -452,6 +510,8 @@ def main():
     from activation_sparse_gemm_b200.inputs import WORKLOADS
     if args.workload == "dit_mlp" and args.impl == "ours":
         return run_block(args)
+    if args.workload == "lora_fit" and args.impl == "ours":
+        return run_lora_fit(args)
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)

@@ -182,3 +182,39 @@ def mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up: int = MO
               mode_down: int = MODE_SPARSE, rows=None):
     return _default().mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up=mode_up,
                                 mode_down=mode_down, rows=rows)
+
+
+# ------------------------------------------------------------------ LoRA fit (closed form)
+def reduced_rank_fit(X: np.ndarray, E: np.ndarray, R: int):
+    """Reduced-rank regression: the rank-R C [N, K] minimising ||X C^T - E||_F,
+    for X [M, K] of full column rank and E [M, N], all float64.
+
+    Least squares B0 = argmin ||X B - E|| (numpy lstsq), the fit Yhat = X B0,
+    its top-R right singular vectors V_R [N, R]; then C^T = B0 V_R V_R^T.
+    Returned as the LoRA factors L_A = V_R [N, R] and L_B = (B0 V_R)^T [R, K]
+    (C = L_A L_B), with the singular values of Yhat."""
+    X = np.asarray(X, np.float64)
+    E = np.asarray(E, np.float64)
+    B0 = np.linalg.lstsq(X, E, rcond=None)[0]
+    _, sig, Vt = np.linalg.svd(X @ B0, full_matrices=False)
+    V = Vt[:R].T
+    return V, (B0 @ V).T, sig
+
+
+def lora_fit(X, W, R: int):
+    """The LoRA of the RT-Lynx summary page's step 2 fitted in closed form on the
+    calibration tokens X (bf16 bits [M, K]): it minimises
+    ||X W^T - S(X) W^T - X (L_A L_B)^T||_F^2, whose target is the residual
+    E = X W^T - S(X) W^T of the dense layer minus the sparse one (both exact,
+    from this oracle).  Returns (L_A float64 [N, R], L_B float64 [R, K], E)."""
+    Yd = linear(X, W, mode=MODE_DENSE_SKIP)
+    Ys = linear(X, W, mode=MODE_SPARSE)
+    E = Yd - Ys
+    L_A, L_B, _ = reduced_rank_fit(bf16_to_f64(X), E, R)
+    return L_A, L_B, E
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns (uint16) to float64, exactly."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -400,3 +400,62 @@ def test_mlp_block_sparse_rows_subset():
     assert (H2 == H[rows]).all() and (Y2 == Y[rows]).all()
     # GELU output is never below its minimum, about -0.17
     assert (bf16_bits_to_f32(H) >= -0.1701).all()
+
+
+# ------------------------------------------------------------------ LoRA fit (reduced-rank regression)
+def _objective(X, E, L_A, L_B):
+    return float(np.linalg.norm(X @ (L_A @ L_B).T - E) ** 2)
+
+
+def test_reduced_rank_fit_recovers_a_planted_map():
+    """E = X C^T with rank(C) = R: the fit returns C exactly (up to rounding)."""
+    rng = np.random.default_rng(11)
+    M, K, N, R = 400, 40, 56, 6
+    X = rng.standard_normal((M, K)) * rng.lognormal(0, 1, K)
+    C = rng.standard_normal((N, R)) @ rng.standard_normal((R, K))
+    L_A, L_B, sig = oracle.reduced_rank_fit(X, X @ C.T, R)
+    assert np.abs(L_A @ L_B - C).max() <= 1e-9 * np.abs(C).max()
+    assert sig[R] <= 1e-9 * sig[0]
+    assert np.allclose(L_A.T @ L_A, np.eye(R), atol=1e-12)
+
+
+def test_reduced_rank_fit_meets_the_eckart_young_optimum():
+    """The objective equals the least-squares residual plus the energy of the
+    discarded singular values of the least-squares fit (the closed-form
+    optimum), falls as R grows, and is below two other rank-R candidates:
+    the truncated SVD of E itself mapped back through least squares, and zero."""
+    rng = np.random.default_rng(12)
+    M, K, N = 300, 32, 48
+    X = rng.standard_normal((M, K))
+    E = rng.standard_normal((M, N)) + X @ rng.standard_normal((K, N))
+    B0 = np.linalg.lstsq(X, E, rcond=None)[0]
+    ls_res = float(np.linalg.norm(X @ B0 - E) ** 2)
+    prev = None
+    for R in (1, 4, 16, 32):
+        L_A, L_B, sig = oracle.reduced_rank_fit(X, E, R)
+        obj = _objective(X, E, L_A, L_B)
+        assert abs(obj - (ls_res + float(np.sum(sig[R:] ** 2)))) <= 1e-9 * obj
+        U, s, Vt = np.linalg.svd(E, full_matrices=False)
+        Et = (U[:, :R] * s[:R]) @ Vt[:R]
+        Bt = np.linalg.lstsq(X, Et, rcond=None)[0]           # a rank-R candidate
+        assert obj <= _objective(X, E, Bt.T, np.eye(K)) * (1 + 1e-12)
+        assert obj <= float(np.linalg.norm(E) ** 2)
+        if prev is not None:
+            assert obj <= prev * (1 + 1e-12)
+        prev = obj
+    assert abs(prev - ls_res) <= 1e-9 * prev  # R = K: the least-squares residual itself
+
+
+def test_lora_fit_targets_the_sparsification_residual():
+    """The fitted LoRA lowers ||X W^T - S(X) W^T - X (L_A L_B)^T||, and with the
+    fitted factors the oracle's layer moves toward the dense layer."""
+    X, W, _, _ = make_custom(700, 64, 48, 8, seed=13, p_out=0.05)
+    R = 8
+    L_A, L_B, E = oracle.lora_fit(X, W, R)
+    Xf = f64(X)
+    assert _objective(Xf, E, L_A, L_B) < 0.95 * float(np.linalg.norm(E) ** 2)
+    A16, B16 = to_bf16_bits(L_A.astype(np.float32)), to_bf16_bits(L_B.astype(np.float32))
+    Yd = oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP)
+    err_none = np.linalg.norm(oracle.linear(X, W) - Yd)
+    err_fit = np.linalg.norm(oracle.linear(X, W, A16, B16) - Yd)
+    assert err_fit < 0.975 * err_none
