@@ -17,11 +17,14 @@
 //         into one of two tensor-memory accumulators.  Where a run crosses a
 //         row block, the partial norms and the partial T of the finished
 //         segment go to the workspace.
-// Pass 2  scale             one warp per token.
-//         Sums the token's partial norms in segment order,
-//         s = ||x|| / (||x~|| + 1e-8) in float, rescales the kept entries in
-//         place (s*x rounded once to bf16, nearest even), and sums the partial
-//         T in segment order, rounded to bf16.
+// Pass 2  scale             eight tokens per CTA, one warp per token for the sums.
+//         Sums each token's partial norms in segment order,
+//         s = ||x|| / (||x~|| + 1e-8) in float, and sums the partial T in
+//         segment order, rounded to bf16; then all threads of the CTA rescale
+//         the kept entries in place (s*x rounded once to bf16, nearest even).
+// Both passes and the GEMM launch as programmatic dependents: each one's setup
+// overlaps the previous kernel's tail, and it touches memory only after the
+// grid-dependency wait.
 // Every reduction runs in a fixed order, so results are deterministic.
 //
 // Metadata chunk (128 tokens x 128 logical K, 2048 bytes), for token m in the

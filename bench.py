@@ -243,7 +243,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     clocks.start()
     # the headline: whole calls, nothing recorded between the kernels (the
-    # GEMM and the scale pass launch as programmatic dependents)
+    # kernels launch as programmatic dependents of one another)
     evs = timed(lambda es: sparse_step(es[0], None, es[1]), args.steps, 2)
     torch.cuda.synchronize()
     clocks.stop()
