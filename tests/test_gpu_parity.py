@@ -274,6 +274,56 @@ def test_full_workload_sampled(name):
         assert_y_close(Yd[rows], oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP, rows=rows), "mlp_down dense")
 
 
+# ------------------------------------------------------------------ workspace and stream contracts
+def test_workspace_contents_need_no_initialisation():
+    """rtlynx_linear_ws on a caller-owned workspace filled with 0xFF bytes
+    (garbage tickets, partials and values) gives the same Y as on a zeroed
+    one, for a shape whose GEMM splits its last tiles along K (tickets)."""
+    import torch
+    M, K, N, R = 4608, 1024, 3072, 64  # 18 row pairs x 13 column tiles: the remainder tiles are split
+    X, W, L_A, L_B = make_custom(M, K, N, R, seed=1201, p_out=0.05)
+    size = rl.rtlynx_workspace_size(M, K, N, R, rl.MODE_SPARSE)
+    outs = []
+    for fill in (0, 0xFF):
+        ws = torch.full((size,), fill, dtype=torch.uint8, device="cuda")
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        rl.rtlynx_linear_ws(dev(X), dev(W), dev(L_A), dev(L_B), Y, M, K, N, R, rl.MODE_SPARSE, ws, size)
+        assert rl.rtlynx_stream_status() == rl.OK
+        outs.append(host_bits(Y))
+    assert (outs[0] == outs[1]).all()
+    rows = [0, 1, 2047, 4607]
+    assert_y_close(outs[1][rows], oracle.linear(X, W, L_A, L_B, rows=rows), "0xFF workspace")
+
+
+def test_two_streams_at_once():
+    """Two different problems queued on two streams without synchronising in
+    between: each stream has its own cached workspace, and both results meet
+    the bar."""
+    import torch
+    probs = [make_custom(1000, 512, 520, 32, seed=1301), make_custom(700, 264, 256, 16, seed=1302)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for (X, W, L_A, L_B), st in zip(probs, streams):  # warm the per-stream workspaces
+        with torch.cuda.stream(st):
+            Y = torch.empty((X.shape[0], W.shape[0]), dtype=torch.bfloat16, device="cuda")
+            rl.rtlynx_linear(dev(X), dev(W), dev(L_A), dev(L_B), Y, X.shape[0], X.shape[1], W.shape[0],
+                             L_B.shape[0], rl.MODE_SPARSE, st)
+    torch.cuda.synchronize()
+    ins = [[dev(a) for a in p] for p in probs]
+    for reps in range(3):
+        outs = []
+        for (Xd, Wd, Ad, Bd), st in zip(ins, streams):
+            with torch.cuda.stream(st):
+                Y = torch.empty((Xd.shape[0], Wd.shape[0]), dtype=torch.bfloat16, device="cuda")
+                rl.rtlynx_linear(Xd, Wd, Ad, Bd, Y, Xd.shape[0], Xd.shape[1], Wd.shape[0], Bd.shape[0],
+                                 rl.MODE_SPARSE, st)
+                outs.append(Y)
+        torch.cuda.synchronize()
+    for (X, W, L_A, L_B), Y in zip(probs, outs):
+        assert_y_close(host_bits(Y), oracle.linear(X, W, L_A, L_B), "two streams", edge=True)
+    assert rl.rtlynx_stream_status(streams[0]) == rl.OK and rl.rtlynx_stream_status(streams[1]) == rl.OK
+
+
 # ------------------------------------------------------------------ host buffers in and out
 @pytest.mark.parametrize("M,K,N,R,mode", [(100, 256, 264, 16, rl.MODE_SPARSE), (3000, 256, 264, 16, rl.MODE_SPARSE),
                                           (5000, 136, 136, 8, rl.MODE_SPARSE), (5000, 136, 136, 8, rl.MODE_DENSE_SKIP)])
