@@ -212,7 +212,13 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
     d.kt2 = 2 * d.k_chunks;
     const int64_t total = d.m_blocks * d.kt2;
     const int64_t sms = num_sms > 0 ? num_sms : 148;
-    d.grid1 = total < sms ? total : sms;
+    // Four tiles a CTA or more once that still leaves 32 CTAs: with fewer, a
+    // row block splits into so many segments that summing their partials
+    // dominates the scale pass.  Very small problems keep a CTA per tile.
+    int64_t by_work = (total + 3) / 4;
+    const int64_t floor_ctas = total < 32 ? total : 32;
+    if (by_work < floor_ctas) by_work = floor_ctas;
+    d.grid1 = by_work < sms ? by_work : sms;
     // A row block's kt2 tiles meet at most (kt2 - 2) / L + 2 runs when every
     // run holds at least L = floor(total / grid1) tiles.
     const int64_t run = total / d.grid1;
