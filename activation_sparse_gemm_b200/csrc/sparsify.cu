@@ -425,11 +425,13 @@ __global__ void __launch_bounds__(256, 4) rtlynx_scale_kernel(const ScaleArgs a)
     }
     __syncthreads();
     for (int i0 = static_cast<int>(threadIdx.x);;) {
+        int r0 = i0 / n16;  // row of the first vector of this round; later ones step it
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const int idx = i0 + 256 * u;
+            while (r0 < kRows - 1 && idx >= (r0 + 1) * n16) ++r0;
             if (idx < total) {
-                const float sr = s_sh[idx / n16];
+                const float sr = s_sh[r0];
                 q[u].x = scale_pair(sr, q[u].x);
                 q[u].y = scale_pair(sr, q[u].y);
                 q[u].z = scale_pair(sr, q[u].z);

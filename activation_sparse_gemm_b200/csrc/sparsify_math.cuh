@@ -4,9 +4,10 @@
 // A group is four consecutive bf16 entries held in two 32-bit words.  The
 // 2-of-4 rule keeps the two largest magnitudes, equal magnitudes going to the
 // lower index.  The prologue ranks each group by the unique key
-// (|x| bits << 2) | (3 - index): integer order of the keys is magnitude order
+// (|x| bits << 16) | (3 - index): integer order of the keys is magnitude order
 // with the lower index winning ties, so the two largest keys are the kept
-// entries.
+// entries.  The magnitude sits where it sits in the high half of the input
+// word, so the keys of odd entries are one mask away from the input.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -20,10 +21,10 @@ struct GroupKeys {
 };
 
 __device__ __forceinline__ GroupKeys rank_group(uint32_t w01, uint32_t w23) {
-    const uint32_t a0 = ((w01 & 0x7FFFu) << 2) | 3u;
-    const uint32_t a1 = ((w01 >> 14) & (0x7FFFu << 2)) | 2u;
-    const uint32_t a2 = ((w23 & 0x7FFFu) << 2) | 1u;
-    const uint32_t a3 = (w23 >> 14) & (0x7FFFu << 2);
+    const uint32_t a0 = ((w01 << 16) & 0x7FFF0000u) | 3u;
+    const uint32_t a1 = (w01 & 0x7FFF0000u) | 2u;
+    const uint32_t a2 = ((w23 << 16) & 0x7FFF0000u) | 1u;
+    const uint32_t a3 = w23 & 0x7FFF0000u;
     const uint32_t h01 = max(a0, a1), l01 = min(a0, a1), h23 = max(a2, a3), l23 = min(a2, a3);
     GroupKeys g;
     g.k1 = max(h01, h23);
@@ -53,15 +54,15 @@ __device__ __forceinline__ uint32_t pick_kept(const GroupKeys& g, uint32_t w01, 
 }
 
 // True when the smallest entry of the group is a normal number (so are the others).
-__device__ __forceinline__ bool group_all_normal(const GroupKeys& g) { return g.k4 >= (0x80u << 2); }
+__device__ __forceinline__ bool group_all_normal(const GroupKeys& g) { return g.k4 >= (0x80u << 16); }
 
 // Adds sum(x^2) of a ranked group whose entries are all normal numbers to
 // `all` and the sum of its two largest squares to `top`.  Each entry is
 // rebuilt as a double from its bits; products of bf16 values are exact in
 // double and each fused multiply-add rounds once.
 __device__ __forceinline__ void group_energy_normal(const GroupKeys& g, double& all, double& top) {
-    const double e1 = bf16_mag_to_double(g.k1 >> 2), e2 = bf16_mag_to_double(g.k2 >> 2);
-    const double e3 = bf16_mag_to_double(g.k3 >> 2), e4 = bf16_mag_to_double(g.k4 >> 2);
+    const double e1 = bf16_mag_to_double(g.k1 >> 16), e2 = bf16_mag_to_double(g.k2 >> 16);
+    const double e3 = bf16_mag_to_double(g.k3 >> 16), e4 = bf16_mag_to_double(g.k4 >> 16);
     const double k = fma(e2, e2, e1 * e1);
     top += k;
     all += fma(e4, e4, fma(e3, e3, k));
@@ -72,8 +73,8 @@ __device__ __forceinline__ void group_energy_normal(const GroupKeys& g, double& 
 // it runs only for the rare tiles that need it, so the common path never pays
 // for its conversions.  Returns (sum of all four squares, sum of the top two).
 static __device__ __noinline__ double2 group_energy_any(uint32_t k1, uint32_t k2, uint32_t k3, uint32_t k4) {
-    const double e1 = __uint_as_float((k1 >> 2) << 16), e2 = __uint_as_float((k2 >> 2) << 16);
-    const double e3 = __uint_as_float((k3 >> 2) << 16), e4 = __uint_as_float((k4 >> 2) << 16);
+    const double e1 = __uint_as_float(k1 & 0x7FFF0000u), e2 = __uint_as_float(k2 & 0x7FFF0000u);
+    const double e3 = __uint_as_float(k3 & 0x7FFF0000u), e4 = __uint_as_float(k4 & 0x7FFF0000u);
     const double k = fma(e2, e2, e1 * e1);
     return make_double2(fma(e4, e4, fma(e3, e3, k)), k);
 }
