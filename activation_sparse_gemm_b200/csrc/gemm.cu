@@ -13,18 +13,20 @@
 // Warp roles in each CTA:
 //   warp 0      TMA producer.  Both CTAs load their halves; the completion of
 //               both is counted on the leader CTA's "full" barrier.  Sparse
-//               stages carry the compressed S(X) tile, the W tile and, every
-//               second stage, one 2 KB metadata chunk; then come the LoRA
-//               stages (T tile and L_A tile).
+//               stages carry the compressed S(X) tile, the W tile and the 2 KB
+//               metadata chunk of their 128 K; then come the LoRA stages (T
+//               tile and L_A tile).
 //   warp 1      tensor-memory owner; in the leader CTA one thread issues every
 //               MMA of the pair: tcgen05.mma.sp (K = 32 logical per instruction)
 //               with the metadata moved into tensor memory by tcgen05.cp, and
 //               dense tcgen05.mma for the LoRA stages into the SAME accumulator,
 //               so T L_A^T never leaves the chip.  Its commits arrive on the
 //               barriers of both CTAs.
-//   warps 2-5   epilogue: tcgen05.ld, optional GELU, round to bf16, swizzled
-//               staging in shared memory, TMA store (clips the ragged M and N
-//               edges).
+//   warps 2-5   epilogue: tcgen05.ld, optional GELU (a template parameter,
+//               used by the feed-forward block's up-projection), round to
+//               bf16; sparse mode stages in swizzled shared memory and stores
+//               by TMA (clipping the ragged M and N edges), dense-skip stores
+//               16-byte pieces straight to Y.
 // The accumulator is double-buffered in tensor memory, so the epilogue of one
 // tile overlaps the main loop of the next.
 //
@@ -40,11 +42,18 @@
 // chain, so its loop only adds precomputed offsets to precomputed
 // descriptors and every stage carries four MMAs per barrier round trip.
 //
-// BN = 240 keeps two accumulators and the metadata inside 512 columns; the
-// epilogue writes it as seven 32-column chunks and one 16-column chunk.
+// Sparse tiles: BN = 240 keeps two accumulators and the metadata inside 512
+// columns; the epilogue writes a tile as seven 32-column chunks and one
+// 16-column chunk.  Dense-skip tiles: BN = 256, two accumulators filling the
+// 512 columns.
 //
 // Tensor memory (per CTA, 512 columns): accumulators at [0, BN) and
-// [BN, 2 BN); metadata of the current 128-wide K chunk at [2 BN, 2 BN + 4).
+// [BN, 2 BN); in sparse mode the metadata of the current 128-wide K chunk at
+// [2 BN, 2 BN + 4).
+//
+// Every launch is a programmatic dependent of the preceding kernel: the setup
+// (barriers, tensor memory, tensor-map prefetch) overlaps that kernel's tail,
+// and operands are read after the grid-dependency wait.
 #include "internal.h"
 #include "ptx.cuh"
 
