@@ -340,8 +340,8 @@ static int run_layer(DeviceInfo* di, const void* X, const void* W, const void* L
     return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
 }
 
-// Which prologue runs: the one-pass cluster kernel (returns its cluster size)
-// or the two-pass path (returns 0).
+// The sparsify prologue: pass 1 and pass 2 (the partition over CTAs is fixed
+// in make_dims).
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
                  cudaStream_t stream) {
     (void)num_sms;  // the split is fixed in make_dims

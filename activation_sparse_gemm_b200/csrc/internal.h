@@ -13,7 +13,6 @@ namespace rtlynx {
 
 // Tile geometry shared by the prologue and the GEMM.
 constexpr int kBM = 128;          // rows (tokens) per tile
-constexpr int kBN = 256;          // output columns per tile
 constexpr int kBK = 64;           // logical K per pipeline stage
 constexpr int kChunkK = 128;      // logical K per metadata chunk (4 sparse MMAs of K = 32)
 constexpr int kChunkBytes = 2048; // 128 lanes x 16 bytes of metadata per chunk
