@@ -307,6 +307,7 @@ def run_ours(args, wl):
     sparse_peak = 2.0 * peaks["bf16_tflops"]
     achieved = gemm_flop / (gemm_mean / 1e3) / 1e12
     traffic = profiled_traffic(wl.name)
+    pro_bytes = 2 * M * K + M * K + M * K // 8 + 4 * M + 2 * M * R + 2 * R * K
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -329,6 +330,13 @@ def run_ours(args, wl):
                      "peak_note": f"2 x {peaks_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s): "
                                   "2:4 sparse nominal ratio"},
         "clocks": clocks.summary(),
+        # the prologue (both passes) against the HBM roofline: algorithmic bytes
+        # are X read, kept values + metadata + s + T written, L_B read once
+        "prologue_roofline": {
+            "bound": "hbm", "bytes": pro_bytes, "achieved": pro_bytes / (statistics.mean(pro_ms) / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": pro_bytes / (statistics.mean(pro_ms) / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "note": "phase time from the split loop (an event between prologue and GEMM)"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
