@@ -132,3 +132,27 @@ def test_block_rejects_bad_arguments():
     with pytest.raises(rl.RtlynxError) as e:  # unknown mode of the second layer
         rl.rtlynx_mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, H, Y, 8, 64, 128, 8, 0, 7)
     assert e.value.status == rl.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("mode_up", [rl.MODE_SPARSE, rl.MODE_DENSE_SKIP])
+@pytest.mark.parametrize("M,D,D_ff,R", [(200, 256, 512, 32), (129, 136, 264, 16), (300, 264, 136, 8),
+                                        (4608, 3072, 12288, 64)])
+def test_block_down_projection_is_the_layer(M, D, D_ff, R, mode_up):
+    """The block's second half is the sparse layer itself, applied to the H
+    the block stores: its Y equals rtlynx_linear on that H, bit for bit
+    (every reduction of the layer runs in a fixed order).  D_ff = 136 gives
+    the down-projection a ragged last metadata chunk; the dense-skip
+    up-projection covers the 256-wide output tiles."""
+    import torch
+    args = make_block_inputs(M, D, D_ff, R, seed=700 + M + D_ff)
+    X, W_up, LA_up, LB_up, W_down, LA_down, LB_down = [dev(a) for a in args]
+    H = torch.empty((M, D_ff), dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    rl.rtlynx_mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, H, Y, M, D, D_ff, R, mode_up,
+                        rl.MODE_SPARSE)
+    Y_layer = torch.empty_like(Y)
+    rl.rtlynx_linear(H, W_down, LA_down, LB_down, Y_layer, M, D_ff, D, R, rl.MODE_SPARSE)
+    assert rl.rtlynx_stream_status() == rl.OK
+    torch.cuda.synchronize()
+    diff = (Y.view(torch.int16) != Y_layer.view(torch.int16))
+    assert not diff.any(), f"{int(diff.sum())} of {diff.numel()} outputs differ"
