@@ -37,8 +37,12 @@ __device__ __forceinline__ GroupKeys rank_group(uint32_t w01, uint32_t w23) {
 
 // A normal bf16 magnitude (exponent field 1..254) as a double, built from its
 // bits: same significand, exponent rebiased from 127 to 1023.  Exact.
-__device__ __forceinline__ double bf16_mag_to_double(uint32_t mag15) {
-    return __hiloint2double(static_cast<int>((mag15 << 13) + ((1023u - 127u) << 20)), 0);
+// From a key (|x| bits << 16 | tag) the high word's significand and exponent
+// bits, mag15 << 13, equal key >> 3 (the tag shifts out); a multiply-high
+// with an added constant forms them on the multiply-add pipe, leaving the
+// integer ALU, which bounds the prologue, to the ranking.
+__device__ __forceinline__ double key_mag_to_double(uint32_t key) {
+    return __hiloint2double(static_cast<int>(__umulhi(key, 1u << 29) + ((1023u - 127u) << 20)), 0);
 }
 
 // The metadata nibble i0 | (i1 << 2) of a ranked group (i0 < i1, the kept
@@ -48,9 +52,10 @@ __device__ __forceinline__ uint32_t pick_kept(const GroupKeys& g, uint32_t w01, 
     const uint32_t ia = (~g.k1) & 3u, ib = (~g.k2) & 3u;  // 3 - (key & 3)
     const uint32_t i0 = min(ia, ib), i1 = max(ia, ib);
     // byte selector picking half-words i0 and i1 out of {w01, w23}
-    const uint32_t sel = (i0 * 0x22u + 0x10u) | ((i1 * 0x22u + 0x10u) << 8);
+    // multiply-adds (the fields do not overlap, so + is |), off the integer ALU
+    const uint32_t sel = i1 * 0x2200u + (i0 * 0x22u + 0x1010u);
     kept = __byte_perm(w01, w23, sel);
-    return i0 | (i1 << 2);
+    return i1 * 4u + i0;
 }
 
 // True when the smallest entry of the group is a normal number (so are the others).
@@ -61,8 +66,8 @@ __device__ __forceinline__ bool group_all_normal(const GroupKeys& g) { return g.
 // rebuilt as a double from its bits; products of bf16 values are exact in
 // double and each fused multiply-add rounds once.
 __device__ __forceinline__ void group_energy_normal(const GroupKeys& g, double& all, double& top) {
-    const double e1 = bf16_mag_to_double(g.k1 >> 16), e2 = bf16_mag_to_double(g.k2 >> 16);
-    const double e3 = bf16_mag_to_double(g.k3 >> 16), e4 = bf16_mag_to_double(g.k4 >> 16);
+    const double e1 = key_mag_to_double(g.k1), e2 = key_mag_to_double(g.k2);
+    const double e3 = key_mag_to_double(g.k3), e4 = key_mag_to_double(g.k4);
     const double k = fma(e2, e2, e1 * e1);
     top += k;
     all += fma(e4, e4, fma(e3, e3, k));
