@@ -8,7 +8,9 @@ triple-loop GEMMs, OpenMP over tokens).  It follows the four-step pipeline
 paragraph of the RT-Lynx summary page (paper.rainbus.top, arXiv 2605.26632),
 steps 1-3: Top-K 2-of-4 mask, norm-compensating scale s, LoRA branch on the
 dense X, and the dense path for skipped layers; plus the feed-forward block of
-two such layers joined by GELU (erf form).  This module only compiles the
+two such layers joined by GELU (erf form), and the layer's FP8 form (E4M3
+codes for W per output channel and for S(X) per token; the reading is in the
+C source).  This module only compiles the
 C file with gcc and marshals numpy arrays through ctypes.
 """
 from __future__ import annotations
@@ -68,6 +70,16 @@ class Oracle:
         lib.oracle_gelu_bf16.restype = ctypes.c_int
         lib.oracle_gelu.argtypes = [ctypes.c_double]
         lib.oracle_gelu.restype = ctypes.c_double
+        lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_quantize_weight_fp8.argtypes = [p, i64, i64, p, p]
+        lib.oracle_quantize_weight_fp8.restype = ctypes.c_int
+        lib.oracle_sparsify_fp8.argtypes = [p, i64, i64, p, p, p, p]
+        lib.oracle_sparsify_fp8.restype = ctypes.c_int
+        lib.oracle_linear_fp8_rows.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, i64, p]
+        lib.oracle_linear_fp8_rows.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         self.lib = lib
@@ -147,6 +159,60 @@ class Oracle:
         Y = self.linear(H, W_down, LA_down, LB_down, mode=mode_down)
         return Y_up, H, Y
 
+    # ------------------------------------------------------------------ FP8 form
+    def e4m3(self, v: float) -> int:
+        """E4M3 code of the float32 value v (nearest, ties to even; saturates at 448)."""
+        return int(self.lib.oracle_e4m3_from_float(float(v)))
+
+    def e4m3_value(self, code: int) -> float:
+        return float(self.lib.oracle_e4m3_to_double(int(code) & 0xFF))
+
+    def quantize_weight_fp8(self, W):
+        """(W8 [N,K] E4M3 codes, q_w [N] float32) for W [N,K] bf16 bits."""
+        W = _u16(W)
+        N, K = W.shape
+        W8 = np.empty((N, K), np.uint8)
+        qw = np.empty((N,), np.float32)
+        if self.lib.oracle_quantize_weight_fp8(_ptr(W), N, K, _ptr(W8), _ptr(qw)):
+            raise ValueError("oracle_quantize_weight_fp8 rejected its arguments")
+        return W8, qw
+
+    def sparsify_fp8(self, X):
+        """Step 1 in FP8: (meta [M,K/4], x8 [M,K/2] E4M3 codes of the kept entries,
+        s [M] float32, q_x [M] float64)."""
+        X = _u16(X)
+        M, K = X.shape
+        meta = np.empty((M, K // 4), np.uint8)
+        x8 = np.empty((M, K // 2), np.uint8)
+        s = np.empty((M,), np.float32)
+        qx = np.empty((M,), np.float64)
+        if self.lib.oracle_sparsify_fp8(_ptr(X), M, K, _ptr(meta), _ptr(x8), _ptr(s), _ptr(qx)):
+            raise ValueError("oracle_sparsify_fp8 rejected its arguments")
+        return meta, x8, s, qx
+
+    def linear_fp8(self, X, W8, qw, L_A=None, L_B=None, rows=None):
+        """Y (float64) of the FP8 form for the listed rows (all when rows is None)."""
+        X = _u16(X)
+        W8 = np.ascontiguousarray(W8, dtype=np.uint8)
+        qw = np.ascontiguousarray(qw, dtype=np.float32)
+        M, K = X.shape
+        N = W8.shape[0]
+        R = 0
+        if L_A is not None and L_B is not None:
+            L_A = _u16(L_A)
+            L_B = _u16(L_B)
+            R = L_B.shape[0]
+        else:
+            L_A = L_B = None
+        rows_arr = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows = M if rows is None else rows_arr.shape[0]
+        Y = np.empty((nrows, N), np.float64)
+        if self.lib.oracle_linear_fp8_rows(_ptr(X), _ptr(W8), _ptr(qw), _ptr(L_A), _ptr(L_B), M, K, N, R,
+                                           _ptr(rows_arr), nrows, _ptr(Y)):
+            raise ValueError("oracle_linear_fp8_rows rejected its arguments")
+        return Y
+
+
 def _default() -> Oracle:
     global _lib
     if _lib is None:
@@ -182,6 +248,26 @@ def mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up: int = MO
               mode_down: int = MODE_SPARSE, rows=None):
     return _default().mlp_block(X, W_up, LA_up, LB_up, W_down, LA_down, LB_down, mode_up=mode_up,
                                 mode_down=mode_down, rows=rows)
+
+
+def e4m3(v: float) -> int:
+    return _default().e4m3(v)
+
+
+def e4m3_value(code: int) -> float:
+    return _default().e4m3_value(code)
+
+
+def quantize_weight_fp8(W):
+    return _default().quantize_weight_fp8(W)
+
+
+def sparsify_fp8(X):
+    return _default().sparsify_fp8(X)
+
+
+def linear_fp8(X, W8, qw, L_A=None, L_B=None, rows=None):
+    return _default().linear_fp8(X, W8, qw, L_A, L_B, rows=rows)
 
 
 # ------------------------------------------------------------------ LoRA fit (closed form)

@@ -225,6 +225,170 @@ int oracle_gelu_bf16(const double *Y, int64_t n, uint16_t *H)
     return 0;
 }
 
+/* ------------------------------------------------------------------ FP8
+ * The FP8 form of the layer (the pages name FP8 as future work that stacks
+ * with the method and give no recipe; the reading, listed in the design
+ * notes):
+ *   - E4M3 is the OCP 8-bit float without infinities (NVIDIA's e4m3): sign,
+ *     4 exponent bits with bias 7, 3 mantissa bits; largest finite magnitude
+ *     448 = 1.75 * 2^8, smallest normal 2^-6, subnormals j * 2^-9 (j = 1..7);
+ *     S.1111.111 is NaN.  Encoding rounds to nearest, ties to even, and
+ *     saturates magnitudes past 448 to 448.
+ *   - W is quantised once per output channel n: B_n = max_k |W[n,k]|,
+ *     w8 = E4M3(W * r_n) with r_n = 448 / B_n, dequantisation scale
+ *     q_w[n] = B_n / 448.
+ *   - S(X) is quantised per token with q_x = max |S(X)| / 448.  s > 0 scales
+ *     every entry of the token alike and the largest |x| is always kept, so
+ *     the codes are E4M3(x~ * r) with r = 448 / A, A = max_k |x_k|, and
+ *     q_x = s * A / 448.
+ *   - The quantisation decisions (r, and the product that is rounded to a
+ *     code) are taken in float32, as a kernel takes them; everything after
+ *     the codes is double.
+ *   - Y = q_x * q_w[n] * sum over kept k of x8 * w8 + T L_A^T, T = X L_B^T
+ *     as in the bf16 form.  An all-zero token or channel has scale 0 and
+ *     codes 0. */
+static uint8_t e4m3_from_double(double v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < 0x1p-6) {
+        /* subnormal range: j * 2^-9, j = 0..8 (j = 8 is 2^-6, code 0x08) */
+        return sign | (uint8_t)nearbyint(ldexp(a, 9));
+    }
+    int e;
+    double m = frexp(a, &e); /* a = m * 2^e, m in [0.5, 1): unbiased exponent e - 1 */
+    int q = (int)nearbyint(ldexp(m, 4)) - 8; /* 3 mantissa bits: 2m in [1, 2) -> 8 + q */
+    int ex = e - 1;
+    if (q == 8) {
+        q = 0;
+        ex += 1;
+    }
+    return sign | (uint8_t)(((ex + 7) << 3) | q);
+}
+
+static double e4m3_to_double(uint8_t c)
+{
+    int ex = (c >> 3) & 0xF, q = c & 7;
+    double a = ex == 0 ? ldexp((double)q, -9) : ldexp(1.0 + q / 8.0, ex - 7);
+    return (c & 0x80) ? -a : a;
+}
+
+uint8_t oracle_e4m3_from_float(float v) { return e4m3_from_double((double)v); }
+double oracle_e4m3_to_double(uint8_t c) { return e4m3_to_double(c); }
+
+/* Per-channel E4M3 weights: W [N,K] bf16 -> W8 [N,K] codes, qw [N] float. */
+int oracle_quantize_weight_fp8(const uint16_t *W, int64_t N, int64_t K, uint8_t *W8, float *qw)
+{
+    if (N < 0 || K <= 0) return 1;
+    for (int64_t n = 0; n < N; ++n) {
+        float b = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = (float)fabs(bf16_to_double(W[n * K + k]));
+            if (a > b) b = a;
+        }
+        float r = b > 0.0f ? 448.0f / b : 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = (float)bf16_to_double(W[n * K + k]) * r;
+            W8[n * K + k] = e4m3_from_double((double)t);
+        }
+        qw[n] = b / 448.0f;
+    }
+    return 0;
+}
+
+/* Step 1 in FP8 for one token: metadata as the bf16 form, the kept entries'
+ * codes x8 [K/2], s, and the token's dequantisation scale q_x (double). */
+static float sparsify_row_fp8(const uint16_t *Xrow, int64_t K, uint8_t *meta, uint8_t *x8, double *qx)
+{
+    float s = sparsify_row(Xrow, K, NULL, NULL, NULL);
+    float A = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = (float)fabs(bf16_to_double(Xrow[k]));
+        if (a > A) A = a;
+    }
+    float r = A > 0.0f ? 448.0f / A : 0.0f;
+    for (int64_t g = 0; g < K / 4; ++g) {
+        double x[4];
+        for (int i = 0; i < 4; ++i) x[i] = bf16_to_double(Xrow[4 * g + i]);
+        int i0, i1;
+        keep_two_of_four(x, &i0, &i1);
+        if (meta) meta[g] = (uint8_t)(i0 | (i1 << 2));
+        x8[2 * g] = e4m3_from_double((double)((float)x[i0] * r));
+        x8[2 * g + 1] = e4m3_from_double((double)((float)x[i1] * r));
+    }
+    *qx = (double)s * (double)A / 448.0;
+    return s;
+}
+
+int oracle_sparsify_fp8(const uint16_t *X, int64_t M, int64_t K, uint8_t *meta, uint8_t *x8, float *s,
+                        double *qx)
+{
+    if (M < 0 || K <= 0 || K % 4) return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t m = 0; m < M; ++m) {
+        double q;
+        float sm = sparsify_row_fp8(X + m * K, K, meta ? meta + m * (K / 4) : NULL, x8 + m * (K / 2), &q);
+        if (s) s[m] = sm;
+        if (qx) qx[m] = q;
+    }
+    return 0;
+}
+
+/* Y rows of the FP8 form for the listed tokens (rows == NULL: all):
+ * Y = q_x q_w[n] sum_{kept k} x8 w8[n,k] + X L_B^T L_A^T.  W8 [N,K] codes,
+ * qw [N] from oracle_quantize_weight_fp8. */
+int oracle_linear_fp8_rows(const uint16_t *X, const uint8_t *W8, const float *qw, const uint16_t *L_A,
+                           const uint16_t *L_B, int64_t M, int64_t K, int64_t N, int64_t R,
+                           const int64_t *rows, int64_t nrows, double *Y)
+{
+    if (M < 0 || K <= 0 || K % 4 || N <= 0 || R < 0) return 1;
+    if (!rows) nrows = M;
+    int use_lora = R > 0 && L_A && L_B;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) {
+            bad = 1;
+            continue;
+        }
+        const uint16_t *Xrow = X + m * K;
+        uint8_t *meta = (uint8_t *)malloc((size_t)(K / 4));
+        uint8_t *x8 = (uint8_t *)malloc((size_t)(K / 2));
+        double *Trow = (double *)malloc(sizeof(double) * (size_t)(R > 0 ? R : 1));
+        double qx;
+        sparsify_row_fp8(Xrow, K, meta, x8, &qx);
+        if (use_lora) {
+            for (int64_t r = 0; r < R; ++r) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += bf16_to_double(Xrow[k]) * bf16_to_double(L_B[r * K + k]);
+                Trow[r] = acc;
+            }
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t g = 0; g < K / 4; ++g) {
+                int i0 = meta[g] & 3, i1 = meta[g] >> 2;
+                acc += e4m3_to_double(x8[2 * g]) * e4m3_to_double(W8[n * K + 4 * g + i0]);
+                acc += e4m3_to_double(x8[2 * g + 1]) * e4m3_to_double(W8[n * K + 4 * g + i1]);
+            }
+            double y = qx * (double)qw[n] * acc;
+            if (use_lora) {
+                double lr = 0.0;
+                for (int64_t r = 0; r < R; ++r) lr += Trow[r] * bf16_to_double(L_A[n * R + r]);
+                y += lr;
+            }
+            Y[i * N + n] = y;
+        }
+        free(meta);
+        free(x8);
+        free(Trow);
+    }
+    return bad ? 1 : 0;
+}
+
 /* Threads the OpenMP runtime will use (reported next to CPU timings). */
 int oracle_num_threads(void)
 {
