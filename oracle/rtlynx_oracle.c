@@ -313,7 +313,7 @@ static float sparsify_row_fp8(const uint16_t *Xrow, int64_t K, uint8_t *meta, ui
         for (int i = 0; i < 4; ++i) x[i] = bf16_to_double(Xrow[4 * g + i]);
         int i0, i1;
         keep_two_of_four(x, &i0, &i1);
-        if (meta) meta[g] = (uint8_t)(i0 | (i1 << 2));
+        if (meta) meta[g] = (uint8_t)((i1 << 2) | i0);
         x8[2 * g] = e4m3_from_double((double)((float)x[i0] * r));
         x8[2 * g + 1] = e4m3_from_double((double)((float)x[i1] * r));
     }
@@ -363,7 +363,7 @@ int oracle_linear_fp8_rows(const uint16_t *X, const uint8_t *W8, const float *qw
             for (int64_t r = 0; r < R; ++r) {
                 double acc = 0.0;
                 for (int64_t k = 0; k < K; ++k)
-                    acc += bf16_to_double(Xrow[k]) * bf16_to_double(L_B[r * K + k]);
+                    acc += bf16_to_double(L_B[r * K + k]) * bf16_to_double(Xrow[k]);
                 Trow[r] = acc;
             }
         }
@@ -377,7 +377,7 @@ int oracle_linear_fp8_rows(const uint16_t *X, const uint8_t *W8, const float *qw
             double y = qx * (double)qw[n] * acc;
             if (use_lora) {
                 double lr = 0.0;
-                for (int64_t r = 0; r < R; ++r) lr += Trow[r] * bf16_to_double(L_A[n * R + r]);
+                for (int64_t r = 0; r < R; ++r) lr += bf16_to_double(L_A[n * R + r]) * Trow[r];
                 y += lr;
             }
             Y[i * N + n] = y;

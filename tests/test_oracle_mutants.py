@@ -55,7 +55,7 @@ PIN_TESTS = [
 def test_pins_catch_mutant(name, tmp_path, monkeypatch):
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    assert src.count(old) == 1, f"mutation site for {name} not found or not unique"
     mut_src = tmp_path / "mutant.c"
     mut_src.write_text(src.replace(old, new))
     lib = oracle.build(force=True, src=str(mut_src), out=str(tmp_path / "libmutant.so"))
