@@ -39,6 +39,7 @@ ABI_SYMBOLS = (
     "rtlynx_workspace_layout",
     "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_mlp_block", "rtlynx_linear_noalloc",
     "rtlynx_kernel_launches",
+    "rtlynx_quantize_weight_fp8", "rtlynx_linear_fp8", "rtlynx_sparsify_fp8_debug",
     "rtlynx_wait_selftest", "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
 )
 
@@ -87,6 +88,12 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_mlp_block.restype = i
         L.rtlynx_linear_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i, p, p]
         L.rtlynx_linear_noalloc.restype = i
+        L.rtlynx_quantize_weight_fp8.argtypes = [p, p, p, p, p, i64, i64, i64, p]
+        L.rtlynx_quantize_weight_fp8.restype = i
+        L.rtlynx_linear_fp8.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p]
+        L.rtlynx_linear_fp8.restype = i
+        L.rtlynx_sparsify_fp8_debug.argtypes = [p, i64, i64, p, p, p, p]
+        L.rtlynx_sparsify_fp8_debug.restype = i
         L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
         L.rtlynx_kernel_launches.restype = i
         L.rtlynx_wait_selftest.argtypes = [i64, p]
@@ -188,6 +195,21 @@ def rtlynx_linear_noalloc(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, dev_status
     device-side timeout code."""
     return _check(lib().rtlynx_linear_noalloc(_ptr(X), _ptr(W), _ptr(L_A), _ptr(L_B), _ptr(Y), M, D_in, D_out, R,
                                               mode, _ptr(dev_status), _stream(stream)), "rtlynx_linear_noalloc")
+
+
+def rtlynx_quantize_weight_fp8(W, L_A, W8, qw, L_A8, D_out, D_in, R, stream=None) -> int:
+    return _check(lib().rtlynx_quantize_weight_fp8(_ptr(W), _ptr(L_A), _ptr(W8), _ptr(qw), _ptr(L_A8), D_out, D_in,
+                                                   R, _stream(stream)), "rtlynx_quantize_weight_fp8")
+
+
+def rtlynx_linear_fp8(X, W8, qw, L_A8, L_B, Y, M, D_in, D_out, R, stream=None) -> int:
+    return _check(lib().rtlynx_linear_fp8(_ptr(X), _ptr(W8), _ptr(qw), _ptr(L_A8), _ptr(L_B), _ptr(Y), M, D_in,
+                                          D_out, R, _stream(stream)), "rtlynx_linear_fp8")
+
+
+def rtlynx_sparsify_fp8_debug(X, M, D_in, codes, meta, qx, stream=None) -> int:
+    return _check(lib().rtlynx_sparsify_fp8_debug(_ptr(X), M, D_in, _ptr(codes), _ptr(meta), _ptr(qx),
+                                                  _stream(stream)), "rtlynx_sparsify_fp8_debug")
 
 
 def rtlynx_kernel_launches(M, D_in, D_out, R, mode) -> int:

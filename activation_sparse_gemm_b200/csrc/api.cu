@@ -196,8 +196,9 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, 
     return 0;
 }
 
-Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
+Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms, bool fp8) {
     Dims d;
+    d.fp8 = fp8;
     d.M = M;
     d.K = K;
     d.N = N;
@@ -227,12 +228,13 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms) {
     // tiles cut along K so that every pair has a part (3 to kMaxSplit parts a
     // tile, each at least two stages long).
     const int64_t m_pairs = d.M_pad / (2 * kBM);
-    const int64_t n_tiles = (N + kPairBN - 1) / kPairBN;
+    const int64_t bn = fp8 ? kFp8BN : kPairBN;
+    const int64_t n_tiles = (N + bn - 1) / bn;
     d.gemm_tiles = m_pairs * n_tiles;
     const int64_t max_pairs = (num_sms > 0 ? num_sms : 148) / 2;
     d.gemm_pairs = d.gemm_tiles < max_pairs ? d.gemm_tiles : max_pairs;
     const int64_t rem = d.gemm_tiles % d.gemm_pairs;
-    const int64_t n_iter = d.k_chunks + d.R_pad / 64;
+    const int64_t n_iter = (fp8 ? d.k_chunks / 2 : d.k_chunks) + d.R_pad / 64;
     int64_t split = rem > 0 ? d.gemm_pairs / rem : 1;
     if (split > kMaxSplit) split = kMaxSplit;
     if (split > n_iter / 2) split = n_iter / 2;
@@ -269,6 +271,13 @@ WsLayout make_ws_layout(const Dims& d) {
     off = align256(off + static_cast<size_t>(d.tail_units) * 2 * kSplitSlotFloats * 4);
     l.split_cnt = off;
     off = align256(off + static_cast<size_t>(d.gemm_tiles - d.tail_full) * 2 * 4);
+    const int64_t f = d.fp8 ? 1 : 0;
+    l.codes = off;
+    off = align256(off + static_cast<size_t>(f * d.M_pad * d.Kc_pad));
+    l.qx = off;
+    off = align256(off + static_cast<size_t>(f * d.M_pad * 4));
+    l.part_amax = off;
+    off = align256(off + static_cast<size_t>(f * d.max_segs * d.M_pad * 4));
     l.total = off;
     return l;
 }
@@ -284,6 +293,9 @@ Workspace carve(void* base, const WsLayout& l) {
     w.part_T = reinterpret_cast<float*>(b + l.part_T);
     w.split_part = reinterpret_cast<float*>(b + l.split_part);
     w.split_cnt = reinterpret_cast<int*>(b + l.split_cnt);
+    w.codes = b + l.codes;
+    w.qx = reinterpret_cast<float*>(b + l.qx);
+    w.part_amax = reinterpret_cast<float*>(b + l.part_amax);
     return w;
 }
 
@@ -476,6 +488,80 @@ int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_i
     if (rc) return rc;
     if (launch_unpack_debug(d, ws, vals, meta, s, R > 0 ? T : nullptr, stream)) return RTLYNX_ERR_CUDA;
     return RTLYNX_OK;
+}
+
+// ---------------------------------------------------------------- FP8 form
+static int validate_fp8(int64_t M, int64_t K, int64_t N, int64_t R) {
+    if (M <= 0 || K <= 0 || N <= 0 || R < 0) return RTLYNX_ERR_INVALID_ARG;
+    if (K % kFp8StageK != 0 || N % 8 != 0) return RTLYNX_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31) - kBM || K > (int64_t(1) << 30) || N > (int64_t(1) << 30))
+        return RTLYNX_ERR_UNSUPPORTED;
+    if (R % 8 != 0 || R > 256) return RTLYNX_ERR_UNSUPPORTED;
+    return RTLYNX_OK;
+}
+
+int rtlynx_quantize_weight_fp8(const void* W, const void* L_A, void* W8, void* qw, void* L_A8, int64_t D_out,
+                               int64_t D_in, int64_t R, void* stream_) {
+    int rc = validate_fp8(1, D_in, D_out, R);
+    if (rc) return rc;
+    if (!W || !W8 || !qw || !aligned16(W) || !aligned16(W8) || !aligned16(qw)) return RTLYNX_ERR_INVALID_ARG;
+    if (R > 0 && (!L_A || !L_A8 || !aligned16(L_A) || !aligned16(L_A8))) return RTLYNX_ERR_INVALID_ARG;
+    DeviceInfo* di = nullptr;
+    rc = current_device(&di);
+    if (rc) return rc;
+    return launch_quantize_weight_fp8(W, R > 0 ? L_A : nullptr, W8, static_cast<float*>(qw), R > 0 ? L_A8 : nullptr,
+                                      D_out, D_in, R, static_cast<cudaStream_t>(stream_))
+               ? RTLYNX_ERR_CUDA
+               : RTLYNX_OK;
+}
+
+int rtlynx_linear_fp8(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B, void* Y,
+                      int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* stream_) {
+    int rc = validate_fp8(M, D_in, D_out, R);
+    if (rc) return rc;
+    if (!X || !W8 || !qw || !Y || !aligned16(X) || !aligned16(W8) || !aligned16(qw) || !aligned16(Y))
+        return RTLYNX_ERR_INVALID_ARG;
+    if (R > 0 && (!L_A8 || !L_B || !aligned16(L_A8) || !aligned16(L_B))) return RTLYNX_ERR_INVALID_ARG;
+    if (Y == X) return RTLYNX_ERR_INVALID_ARG;
+    DeviceInfo* di = nullptr;
+    rc = current_device(&di);
+    if (rc) return rc;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const Dims d = make_dims(M, D_in, D_out, R, di->num_sms, true);
+    const WsLayout l = make_ws_layout(d);
+    void* base = nullptr;
+    rc = cached_workspace(dev, stream, l.total, &base);
+    if (rc) return rc;
+    const Workspace ws = carve(base, l);
+    const bool lora = R > 0;
+    if (launch_sparsify(d, X, lora ? L_B : nullptr, ws, di->err_word, stream)) return RTLYNX_ERR_CUDA;
+    if (launch_gemm(d, true, nullptr, W8, lora ? L_A8 : nullptr, ws, Y, 0, di->num_sms, di->err_word, stream,
+                    static_cast<const float*>(qw)))
+        return RTLYNX_ERR_CUDA;
+    return RTLYNX_OK;
+}
+
+int rtlynx_sparsify_fp8_debug(const void* X, int64_t M, int64_t D_in, void* codes, void* meta, void* qx,
+                              void* stream_) {
+    int rc = validate_fp8(M, D_in, 8, 0);
+    if (rc) return rc;
+    if (!X || !aligned16(X)) return RTLYNX_ERR_INVALID_ARG;
+    DeviceInfo* di = nullptr;
+    rc = current_device(&di);
+    if (rc) return rc;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const Dims d = make_dims(M, D_in, 8, 0, di->num_sms, true);
+    const WsLayout l = make_ws_layout(d);
+    void* base = nullptr;
+    rc = cached_workspace(dev, stream, l.total, &base);
+    if (rc) return rc;
+    const Workspace ws = carve(base, l);
+    if (launch_sparsify(d, X, nullptr, ws, di->err_word, stream)) return RTLYNX_ERR_CUDA;
+    return launch_unpack_fp8_debug(d, ws, codes, meta, qx, stream) ? RTLYNX_ERR_CUDA : RTLYNX_OK;
 }
 
 int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const void* L_B, void* Y_host,

@@ -63,14 +63,17 @@ constexpr int kPairThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kEpiBufBytes = 32 * 64;  // one warp's 32 rows x 32 bf16 columns
 
-template <bool SPARSE, int BN>
+// FP8: E4M3 operands; a stage of 256 logical K has the bf16 sparse stage's
+// A and B bytes (128-byte rows) and two metadata chunks.
+template <bool SPARSE, int BN, bool FP8 = false>
 struct PairShape {
     static constexpr int BN_HALF = BN / 2;
-    static constexpr int BK = SPARSE ? 128 : 64;                 // logical K per stage
+    static constexpr int BK = FP8 ? kFp8StageK : (SPARSE ? 128 : 64);  // logical K per stage
     static constexpr int A_BYTES = kBM * 64 * 2;                  // 128 rows x 128 B
     static constexpr int B_ATOM_BYTES = BN_HALF * 64 * 2;        // BN/2 rows x 128 B
-    static constexpr int B_BYTES = (BK / 64) * B_ATOM_BYTES;
-    static constexpr int E_BYTES = SPARSE ? kChunkBytes : 0;
+    static constexpr int B_BYTES = (FP8 ? 2 : BK / 64) * B_ATOM_BYTES;
+    static constexpr int E_CHUNKS = SPARSE ? (FP8 ? 2 : 1) : 0;  // metadata chunks (128 logical K each) per stage
+    static constexpr int E_BYTES = E_CHUNKS * kChunkBytes;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
     static constexpr int STAGES = SPARSE ? 4 : 6;
     static constexpr int LORA_A_BYTES = kBM * 64 * 2;
@@ -78,7 +81,7 @@ struct PairShape {
     static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-    static_assert(BN % 16 == 0 && BN >= 64 && 2 * BN + (SPARSE ? 4 : 0) <= 512,
+    static_assert(BN % (FP8 ? 32 : 16) == 0 && BN >= 64 && 2 * BN + 4 * E_CHUNKS <= 512,
                   "two accumulators (and, when sparse, the metadata) must fit");
     static_assert(B_ATOM_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
     static_assert(LORA_A_BYTES <= A_BYTES && LORA_B_BYTES <= B_BYTES, "LoRA tiles must fit the operand slots");
@@ -99,6 +102,8 @@ struct PairArgs {
     float* split_part;  // fp32 partial tile of each part, per CTA of the pair
     int* split_cnt;     // arrival ticket of each split tile, per CTA of the pair (zeroed by the prologue)
     uint16_t* Y;        // [M, N] bf16 output, row-major (the dense-skip epilogue stores to it directly)
+    const float* qx;    // FP8: [M_pad] per-token scale
+    const float* qw;    // FP8: [N] per-channel scale (0 for an all-zero channel, applied as 1)
     int* err;
 };
 
@@ -208,13 +213,13 @@ __device__ __forceinline__ void store_row_bf16(const PairArgs& a, int row, int c
     }
 }
 
-template <bool SPARSE, int BN, int ACT>
+template <bool SPARSE, int BN, int ACT, bool FP8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     rtlynx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmLA,
                             const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                             const __grid_constant__ CUtensorMap tmY16, const PairArgs args) {
-    using G = PairShape<SPARSE, BN>;
+    using G = PairShape<SPARSE, BN, FP8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi = smem + G::STAGES * G::STAGE_BYTES;
@@ -303,11 +308,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const uint32_t fbar = full0 + static_cast<uint32_t>(stage) * 8u;
                     if (kt < args.k_stages) {
                         if (leader) mbar_arrive_expect_tx(&full[stage], 2u * (G::A_BYTES + G::B_BYTES + G::E_BYTES));
-                        tma_load_2d_pair(sA, &tmA, fbar, kt * 64, row0);
+                        // A and B coordinates count elements: 128-byte rows hold 64 bf16 or 128 E4M3
+                        constexpr int kRowElems = FP8 ? 128 : 64;
+                        tma_load_2d_pair(sA, &tmA, fbar, kt * kRowElems, row0);
                         tma_load_2d_pair(sB, &tmB, fbar, kt * G::BK, col0);
                         if constexpr (SPARSE) {
-                            tma_load_2d_pair(sB + G::B_ATOM_BYTES, &tmB, fbar, kt * G::BK + 64, col0);
-                            tma_load_2d_pair(sB + G::B_BYTES, &tmE, fbar, 0, (chunk0 + kt) * 4);
+                            tma_load_2d_pair(sB + G::B_ATOM_BYTES, &tmB, fbar, kt * G::BK + kRowElems, col0);
+                            tma_load_2d_pair(sB + G::B_BYTES, &tmE, fbar, 0, (chunk0 + kt * G::E_CHUNKS) * 4);
                         }
                     } else {
                         const int j = kt - args.k_stages;
@@ -333,7 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
     } else if (warp == 1) {
         if (leader && lane == 0) {
-            const uint32_t idesc_main = make_idesc_bf16(2 * kBM, BN, SPARSE);
+            const uint32_t idesc_main = FP8 ? make_idesc_e4m3(2 * kBM, BN, true) : make_idesc_bf16(2 * kBM, BN, SPARSE);
             const uint32_t idesc_dense = make_idesc_bf16(2 * kBM, BN, false);
             // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the
             // start-address field, operand offsets inside a stage likewise.
@@ -369,7 +376,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const uint64_t b = descB0 + off;
                     const uint32_t acc = kt != w.kb;  // the item's first stage starts the accumulator
                     if (kt < args.k_stages) {
-                        if constexpr (SPARSE) {
+                        if constexpr (FP8) {
+                            // two metadata chunks -> columns [meta, meta + 8); MMA j reads columns meta + 2j, + 2j + 1
+                            tmem_cp_128x128b_pair(tmem_meta, descE0 + off);
+                            tmem_cp_128x128b_pair(tmem_meta + 4u, descE0 + off + (kChunkBytes >> 4));
+                            mma_sp_f8_pair(d, a, b, tmem_meta, idesc_main, acc);
+                            mma_sp_f8_pair(d, a + 2, b + 4, tmem_meta + 2u, idesc_main, 1u);
+                            mma_sp_f8_pair(d, a + 4, b + kAtomStep, tmem_meta + 4u, idesc_main, 1u);
+                            mma_sp_f8_pair(d, a + 6, b + kAtomStep + 4, tmem_meta + 6u, idesc_main, 1u);
+                        } else if constexpr (SPARSE) {
                             tmem_cp_128x128b_pair(tmem_meta, descE0 + off);
                             mma_sp_f16_pair(d, a, b, e01, id0, acc);
                             mma_sp_f16_pair(d, a + 2, b + 4, e01, id1, 1u);
@@ -538,6 +553,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                             }
                         }
                     }
+                    if constexpr (FP8) {  // dequantise: q_x of the token times q_w of the column
+                        const float qxr = args.qx[row0 + lane];
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) {
+                            const int col = col0 + c + q;
+                            float w = col < args.N ? args.qw[col] : 1.0f;
+                            w = w > 0.0f ? w : 1.0f;
+                            r[q] = __float_as_uint(__uint_as_float(r[q]) * (qxr * w));
+                        }
+                    }
                     if constexpr (ACT == 1) {
 #pragma unroll
                         for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(gelu_erf(__uint_as_float(r[q])));
@@ -606,12 +631,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
 }
 
-template <bool SPARSE, int BN, int ACT>
+template <bool SPARSE, int BN, int ACT, bool FP8 = false>
 static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmT,
                        const CUtensorMap& tmLA, const CUtensorMap& tmE, const CUtensorMap& tmY,
                        const CUtensorMap& tmY16, const PairArgs& args, int num_sms, cudaStream_t stream) {
-    using G = PairShape<SPARSE, BN>;
-    auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN, ACT>;
+    using G = PairShape<SPARSE, BN, FP8>;
+    auto kernel = rtlynx_gemm_pair_kernel<SPARSE, BN, ACT, FP8>;
     static std::atomic<uint64_t> smem_set{0};
     const int e = allow_max_dynamic_smem(kernel, smem_set);
     if (e) return e;
@@ -626,14 +651,25 @@ static int launch_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUt
 }
 
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
-                void* Y, int act, int num_sms, int* err, cudaStream_t stream) {
+                void* Y, int act, int num_sms, int* err, cudaStream_t stream, const float* qw) {
     // Sparse tiles are 240 wide so that two accumulators and the metadata fit
     // in 512 tensor-memory columns; dense-skip tiles carry no metadata and are
     // 256 wide (two accumulators fill the 512 columns).
-    const int BN = sparse ? kPairBN : kDenseBN;
+    const bool fp8 = sparse && d.fp8;
+    if (fp8 && (act != 0 || !qw || d.K % kFp8StageK)) return static_cast<int>(cudaErrorInvalidValue);
+    const int BN = fp8 ? kFp8BN : (sparse ? kPairBN : kDenseBN);
     CUtensorMap tmA, tmB, tmT, tmLA, tmE, tmY, tmY16;
     int rc;
-    if (sparse) {
+    if (fp8) {
+        // E4M3 codes of the kept entries and of W (one byte each), 128-byte boxes
+        rc = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.codes, d.Kc_pad, d.M_pad, d.Kc_pad, 128, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc) return rc;
+        // two metadata chunks per stage: eight rows of 256 16-bit words
+        rc = encode_tmap_2d(&tmE, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, ws.meta, 256, d.m_blocks * d.k_chunks * 4, 512,
+                            256, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc) return rc;
+    } else if (sparse) {
         rc = encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.vals, d.Kc_pad, d.M_pad, d.Kc_pad * 2,
                             64, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc) return rc;
@@ -647,8 +683,10 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
         if (rc) return rc;
         tmE = tmA;
     }
-    rc = encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, d.K, d.N, d.K * 2, kBK, BN / 2,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+    rc = fp8 ? encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, W, d.K, d.N, d.K, 128, BN / 2,
+                              CU_TENSOR_MAP_SWIZZLE_128B)
+             : encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, d.K, d.N, d.K * 2, kBK, BN / 2,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     rc = encode_tmap_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d.N, d.M, d.N * 2, 32, 32,
                         CU_TENSOR_MAP_SWIZZLE_64B);
@@ -673,7 +711,7 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.N = static_cast<int>(d.N);
     args.m_pairs = static_cast<int>((d.M + 2 * kBM - 1) / (2 * kBM));
     args.n_tiles = static_cast<int>((d.N + BN - 1) / BN);
-    args.k_stages = static_cast<int>(sparse ? d.k_chunks : d.k_tiles);
+    args.k_stages = static_cast<int>(fp8 ? d.k_chunks / 2 : (sparse ? d.k_chunks : d.k_tiles));
     args.lora_stages = lora ? static_cast<int>(d.R_pad / 64) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
     {
@@ -703,7 +741,10 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.split_part = ws.split_part;
     args.split_cnt = ws.split_cnt;
     args.Y = static_cast<uint16_t*>(Y);
+    args.qx = ws.qx;
+    args.qw = qw;
     args.err = err;
+    if (fp8) return launch_pair<true, kFp8BN, 0, true>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream);
     // the epilogue activation is a template parameter, so the plain kernels carry no GELU code
     if (act == 1)
         return sparse ? launch_pair<true, kPairBN, 1>(tmA, tmB, tmT, tmLA, tmE, tmY, tmY16, args, num_sms, stream)

@@ -18,6 +18,11 @@ constexpr int kChunkK = 128;      // logical K per metadata chunk (4 sparse MMAs
 constexpr int kChunkBytes = 2048; // 128 lanes x 16 bytes of metadata per chunk
 constexpr int kPairBN = 240;      // output columns per sparse GEMM tile (one CTA pair)
 constexpr int kDenseBN = 256;     // output columns per dense-skip GEMM tile
+// FP8 (E4M3) sparse tiles: the f8f6f4 sparse MMA of a CTA pair wants N a
+// multiple of 32, and two accumulators plus eight metadata columns must fit
+// in 512; a stage carries 256 logical K (the same bytes as a bf16 stage).
+constexpr int kFp8BN = 224;
+constexpr int kFp8StageK = 256;
 // fp32 partial of one CTA's 128 x 240 tile: [32-column chunk 8][4-column group 8][row 128][4]
 constexpr int kSplitSlotFloats = 8 * kBM * 32;
 constexpr int kMaxSplit = 6;  // parts of one split tile (the fix-up holds two chunks of the others in shared memory)
@@ -38,6 +43,7 @@ struct Dims {
     // `tail_full` tiles round-robin; each of the remaining tiles is cut along K
     // into `tail_split` parts, one per pair (`tail_units` parts in all).
     int64_t gemm_pairs, gemm_tiles, tail_full, tail_split, tail_units;
+    bool fp8;             // the FP8 form: E4M3 codes, 224-wide tiles, 256-K stages
 };
 
 // The streaming prologue cuts the m_blocks * kt2 tiles into `grid` contiguous
@@ -50,10 +56,12 @@ __host__ __device__ inline int64_t stream_owner(int64_t t, int64_t total, int64_
 
 // Byte offsets of the sparse-mode workspace regions (each 256-byte aligned).
 struct WsLayout {
-    size_t vals, meta, s, T, part_norm, part_T, split_part, split_cnt, total;
+    size_t vals, meta, s, T, part_norm, part_T, split_part, split_cnt;
+    size_t codes, qx, part_amax;  // FP8 form only (empty otherwise)
+    size_t total;
 };
 
-Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms);
+Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms, bool fp8 = false);
 WsLayout make_ws_layout(const Dims& d);
 
 struct Workspace {
@@ -65,6 +73,11 @@ struct Workspace {
     float* part_T;        // [max_segs, M_pad, R_pad] partial X L_B^T
     float* split_part;    // [tail_units, 2, kSplitSlotFloats] fp32 partial tiles of the split tail
     int* split_cnt;       // [2 * (gemm_tiles - tail_full)] arrival tickets of the split tiles
+    // FP8 form: metadata in the 8-bit layout (row m of a 128-token block at
+    // byte 16 m of each 2 KB chunk, group g at nibble g of the row's 16 bytes)
+    uint8_t* codes;       // [M_pad, Kc_pad] E4M3 codes of the kept entries
+    float* qx;            // [M_pad] per-token dequantisation scale s * max|x| / 448
+    float* part_amax;     // [max_segs, M_pad] partial max |x|
 };
 
 // Tensor-map encoding through the driver entry point (no libcuda link needed).
@@ -119,7 +132,13 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
                     cudaStream_t stream);
 // act: 0 none, 1 GELU (erf form) applied to the output before its bf16 rounding.
 int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const void* L_A, const Workspace& ws,
-                void* Y, int act, int num_sms, int* err, cudaStream_t stream);
+                void* Y, int act, int num_sms, int* err, cudaStream_t stream, const float* qw = nullptr);
+// FP8 weight preparation: W8 = E4M3(W * 448 / max|W_n|), qw = max|W_n| / 448,
+// L_A8 = L_A / qw (rows of all-zero channels divided by 1).
+int launch_quantize_weight_fp8(const void* W, const void* L_A, void* W8, float* qw, void* L_A8, int64_t N,
+                               int64_t K, int64_t R, cudaStream_t stream);
+int launch_unpack_fp8_debug(const Dims& d, const Workspace& ws, void* codes, void* meta, void* qx,
+                            cudaStream_t stream);
 // Shared by the entry points (api.cu).
 bool ensure_tmap_encoder();
 Workspace carve(void* base, const WsLayout& l);

@@ -337,6 +337,18 @@ __device__ __forceinline__ void mma_sp_f16_pair(uint32_t d_tmem, uint64_t a_desc
         : "memory");
 }
 
+// The same for E4M3 operands (K = 64 logical per instruction); the metadata
+// of the 64 K sits in two consecutive tensor-memory columns from e_tmem (even).
+__device__ __forceinline__ void mma_sp_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
@@ -364,6 +376,13 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool sparse
            | (1u << 4)                    // D format: f32
            | (1u << 7)                    // A format: bf16
            | (1u << 10)                   // B format: bf16
+           | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// E4M3 x E4M3 -> f32 (kind::f8f6f4: A and B format 0 = E4M3).
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N, bool sparse) {
+    return (sparse ? (1u << 2) : 0u)      // sparsity enable
+           | (1u << 4)                    // D format: f32
            | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -33,6 +33,8 @@
 //     tensor-memory lane dp = m0 + 8*k1 + 16*m2, column k2,
 //     byte offset 16*dp + 4*k2, bit 16*m1 + 4*(k0 / 4) within that 32-bit word,
 // and the nibble of a group is i0 | (i1 << 2) with i0 < i1 the kept indices.
+#include <cuda_fp8.h>
+
 #include "internal.h"
 #include "ptx.cuh"
 #include "sparsify_math.cuh"
@@ -50,6 +52,7 @@ struct StreamArgs {
     uint8_t* meta;
     double* part_norm;
     float* part_T;
+    float* part_amax;  // FP8 form: [max_segs, M_pad] partial max |x|
     int* split_cnt;  // arrival tickets of the GEMM's split tiles, zeroed here for the GEMM that follows
     int n_split_cnt;
     int* err;
@@ -74,7 +77,10 @@ __device__ __forceinline__ int64_t stream_owner_dev(int64_t t, int64_t total, in
     return static_cast<int64_t>(num / static_cast<uint64_t>(total));
 }
 
-template <bool LORA>
+// FP8: the metadata goes out in the 8-bit layout (token m of the block at
+// byte 16 m of each chunk, group g of the chunk at nibble g), and each
+// segment's max |x| per token goes to part_amax.
+template <bool LORA, bool FP8>
 __global__ void __launch_bounds__(kStreamThreads, 1)
     rtlynx_sparsify_stream_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmLB,
                                   const StreamArgs a) {
@@ -239,6 +245,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
             uint16_t* vB = vA + 8 * a.Kc_pad;
             uint8_t* mrow = a.meta + mb * a.k_chunks * kChunkBytes + dp * 16;
             double nxA = 0.0, ntA = 0.0, nxB = 0.0, ntB = 0.0;
+            uint32_t mkA = 0u, mkB = 0u;  // FP8: the largest key of each token's entries in this segment
+            uint8_t* mchunk8 = a.meta + mb * a.k_chunks * kChunkBytes;
             bool ok = true;
             for (int kt = static_cast<int>(t - mb * kt2); t < seg_end; ++t, ++kt) {
                 if (!warp_wait(&full[stage], phase, err)) {
@@ -283,12 +291,21 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 }
                 *reinterpret_cast<uint2*>(vA + kt * 32) = ka;
                 *reinterpret_cast<uint2*>(vB + kt * 32) = kb;
-                // metadata word: bytes (rA, u even), (rA, u odd), (rB, u even), (rB, u odd)
-                const uint32_t mine = na | (nb << 8);
-                const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
-                if (even)
-                    *reinterpret_cast<uint32_t*>(mrow + (kt >> 1) * kChunkBytes + (2 * (kt & 1) + (u >> 2)) * 4) =
-                        __byte_perm(mine, other, 0x5140);
+                if constexpr (FP8) {
+                    mkA = max(mkA, max(g0.k1, g1.k1));
+                    mkB = max(mkB, max(g2.k1, g3.k1));
+                    // one byte (groups 2u and 2u + 1 of this 64-wide tile) per token
+                    uint8_t* c8 = mchunk8 + (kt >> 1) * kChunkBytes + (kt & 1) * 8 + u;
+                    c8[16 * rA] = static_cast<uint8_t>(na);
+                    c8[16 * (rA + 8)] = static_cast<uint8_t>(nb);
+                } else {
+                    // metadata word: bytes (rA, u even), (rA, u odd), (rB, u even), (rB, u odd)
+                    const uint32_t mine = na | (nb << 8);
+                    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
+                    if (even)
+                        *reinterpret_cast<uint32_t*>(mrow + (kt >> 1) * kChunkBytes + (2 * (kt & 1) + (u >> 2)) * 4) =
+                            __byte_perm(mine, other, 0x5140);
+                }
             }
             if (!ok) break;
             // the token's totals over the eight units, in a fixed order
@@ -298,6 +315,17 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 ntA += __shfl_xor_sync(0xFFFFFFFFu, ntA, o);
                 nxB += __shfl_xor_sync(0xFFFFFFFFu, nxB, o);
                 ntB += __shfl_xor_sync(0xFFFFFFFFu, ntB, o);
+            }
+            if constexpr (FP8) {
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    mkA = max(mkA, __shfl_xor_sync(0xFFFFFFFFu, mkA, o));
+                    mkB = max(mkB, __shfl_xor_sync(0xFFFFFFFFu, mkB, o));
+                }
+                if (u == 0) {  // the key's high half is the bf16 magnitude: as a float, |x| exactly
+                    a.part_amax[seg * a.M_pad + growA] = __uint_as_float(mkA & 0x7FFF0000u);
+                    a.part_amax[seg * a.M_pad + growA + 8] = __uint_as_float(mkB & 0x7FFF0000u);
+                }
             }
             if (u == 0) {
                 double* pn = a.part_norm + (seg * a.M_pad + growA) * 2;
@@ -350,6 +378,10 @@ struct ScaleArgs {
     uint16_t* vals;
     float* s_out;
     uint16_t* T;
+    // FP8 form
+    const float* part_amax;
+    uint8_t* codes;
+    float* qx;
 };
 
 // Eight tokens per CTA (all in one row block, so they share the segment
@@ -358,11 +390,16 @@ struct ScaleArgs {
 // token's partial norms (one segment per lane) and partial T (up to four
 // segments at a time).  Warp w then forms token w's s and T; after one CTA
 // barrier all 256 threads rescale the span.
+// FP8: instead of the in-place rescale, the kept entries become E4M3 codes of
+// x * (448 / max|x|) (float32 product, nearest even, saturating), the token's
+// dequantisation scale q_x = s * max|x| / 448 is stored, and T is stored as
+// T / q_x (the GEMM multiplies its accumulator by q_x q_w).
+template <bool FP8>
 __global__ void __launch_bounds__(256, 4) rtlynx_scale_kernel(const ScaleArgs a) {
     constexpr int kRows = 8;  // tokens per CTA
     constexpr int kU = 8;     // 16-byte value vectors in flight per thread
     constexpr int kSegU = 4;  // partial-T segments loaded at once
-    __shared__ float s_sh[kRows];
+    __shared__ float s_sh[kRows];  // s, or with FP8 the code scale 448 / max|x|
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
     const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;  // M_pad is a multiple of kRows
@@ -384,7 +421,37 @@ __global__ void __launch_bounds__(256, 4) rtlynx_scale_kernel(const ScaleArgs a)
         if (static_cast<int>(threadIdx.x) + 256 * u < total) q[u] = v[threadIdx.x + 256 * u];
     double2 part = make_double2(0.0, 0.0);
     if (lane < nseg) part = *reinterpret_cast<const double2*>(a.part_norm + (lane * a.M_pad + row) * 2);
-    // T needs no s: partial sums in segment order, rounded once to bf16
+    float amax = 0.0f, inv_q = 1.0f, code_scale = 0.0f;
+    if constexpr (FP8) {
+        for (int j = lane; j < nseg; j += 32) amax = fmaxf(amax, a.part_amax[j * a.M_pad + row]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        // s first: q_x needs it before T is stored
+        double nx = 0.0, nt = 0.0;
+        for (int j0 = 0; j0 < nseg; j0 += 32) {
+            double2 p2 = part;
+            if (j0 > 0) {
+                p2 = make_double2(0.0, 0.0);
+                if (j0 + lane < nseg)
+                    p2 = *reinterpret_cast<const double2*>(a.part_norm + ((j0 + lane) * a.M_pad + row) * 2);
+            }
+            const int m = nseg - j0 < 32 ? nseg - j0 : 32;
+            for (int j = 0; j < m; ++j) {
+                nx += __shfl_sync(0xFFFFFFFFu, p2.x, j);
+                nt += __shfl_sync(0xFFFFFFFFu, p2.y, j);
+            }
+        }
+        const float s = static_cast<float>(sqrt(nx) / (sqrt(nt) + 1e-8));
+        const float q = __fdiv_rn(__fmul_rn(s, amax), 448.0f);
+        inv_q = q > 0.0f ? __fdiv_rn(1.0f, q) : 0.0f;
+        code_scale = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
+        if (lane == 0) {
+            s_sh[w] = code_scale;
+            a.s_out[row] = s;
+            a.qx[row] = q;
+        }
+    }
+    // T: partial sums in segment order, rounded once to bf16 (with FP8, T / q_x)
     for (int c = 2 * lane; c < a.R_pad; c += 64) {
         float t0 = 0.f, t1 = 0.f;
         for (int j0 = 0; j0 < nseg; j0 += kSegU) {
@@ -401,7 +468,43 @@ __global__ void __launch_bounds__(256, 4) rtlynx_scale_kernel(const ScaleArgs a)
                 }
             }
         }
+        if (FP8) {
+            t0 *= inv_q;
+            t1 *= inv_q;
+        }
         *reinterpret_cast<__nv_bfloat162*>(a.T + row * a.R_pad + c) = __floats2bfloat162_rn(t0, t1);
+    }
+    if constexpr (FP8) {
+        __syncthreads();
+        // codes of the CTA's span: 8 kept entries (one 16-byte vector) -> 8 bytes
+        uint2* out = reinterpret_cast<uint2*>(a.codes + row0 * a.Kc_pad);
+        for (int i0 = static_cast<int>(threadIdx.x);;) {
+            int r0 = i0 / n16;
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int idx = i0 + 256 * u;
+                while (r0 < kRows - 1 && idx >= (r0 + 1) * n16) ++r0;
+                if (idx < total) {
+                    const float cs = s_sh[r0];
+                    const uint32_t wv[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+                    uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float lo = __fmul_rn(__uint_as_float(wv[h] << 16), cs);
+                        const float hi = __fmul_rn(__uint_as_float(wv[h] & 0xFFFF0000u), cs);
+                        const uint32_t c2 = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+                        pk[h >> 1] |= c2 << (16 * (h & 1));
+                    }
+                    out[idx] = make_uint2(pk[0], pk[1]);
+                }
+            }
+            i0 += 256 * kU;
+            if (i0 >= total) break;
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                if (i0 + 256 * u < total) q[u] = v[i0 + 256 * u];
+        }
+        return;
     }
     // partial norms, one segment per lane, added in segment order (every lane
     // forms the same s)
@@ -493,6 +596,7 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
         tmLB = tmX;
     }
     StreamArgs a;
+    a.part_amax = ws.part_amax;
     a.M_pad = d.M_pad;
     a.Kc_pad = d.Kc_pad;
     a.total_tiles = d.m_blocks * d.kt2;
@@ -512,9 +616,10 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
     const int smem = a.stages * stage_bytes + 256 + 1024;
     const dim3 grid(static_cast<unsigned>(d.grid1));
     cudaError_t e;
-    static std::atomic<uint64_t> smem_set[2];
-    auto kernel = lora ? rtlynx_sparsify_stream_kernel<true> : rtlynx_sparsify_stream_kernel<false>;
-    const int rc2 = allow_max_dynamic_smem(kernel, smem_set[lora ? 1 : 0]);
+    static std::atomic<uint64_t> smem_set[4];
+    auto kernel = d.fp8 ? (lora ? rtlynx_sparsify_stream_kernel<true, true> : rtlynx_sparsify_stream_kernel<false, true>)
+                        : (lora ? rtlynx_sparsify_stream_kernel<true, false> : rtlynx_sparsify_stream_kernel<false, false>);
+    const int rc2 = allow_max_dynamic_smem(kernel, smem_set[(lora ? 1 : 0) + (d.fp8 ? 2 : 0)]);
     if (rc2) return rc2;
     e = static_cast<cudaError_t>(launch_dependent(kernel, grid, dim3(kStreamThreads), smem, stream, tmX, tmLB, a));
     if (e != cudaSuccess) return e;
@@ -535,7 +640,10 @@ int launch_sparsify(const Dims& d, const void* X, const void* L_B, const Workspa
     b.vals = ws.vals;
     b.s_out = ws.s;
     b.T = ws.T;
-    return launch_dependent(rtlynx_scale_kernel, dim3(static_cast<unsigned>(d.M_pad / 8)), dim3(256), 0, stream, b);
+    b.part_amax = ws.part_amax;
+    b.codes = ws.codes;
+    b.qx = ws.qx;
+    return launch_dependent(d.fp8 ? rtlynx_scale_kernel<true> : rtlynx_scale_kernel<false>, dim3(static_cast<unsigned>(d.M_pad / 8)), dim3(256), 0, stream, b);
 }
 
 int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,

@@ -109,6 +109,38 @@ int rtlynx_workspace_layout(int64_t M, int64_t D_in, int64_t D_out, int64_t R, r
 int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_in, int64_t R, void* vals,
                           void* meta, void* s, void* T, void* stream);
 
+/* ---------------------------------------------------------------- FP8 form
+ * The layer with E4M3 operands (the pages name FP8 as future work that
+ * stacks with the method; the recipe is this library's reading):
+ *   - W per output channel: qw[n] = max_k |W[n,k]| / 448 and codes
+ *     W8 = E4M3(W * 448 / max|W_n|), float32 product, nearest even,
+ *     saturating at 448; all-zero channels get qw = 0 and zero codes;
+ *   - S(X) per token: q_x = s * max|x| / 448, codes of the kept entries
+ *     E4M3(x~ * 448 / max|x|) (the largest |x| of a token is always kept);
+ *   - Y = q_x qw[n] sum(x8 w8) + X L_B^T L_A^T, rounded to bf16.
+ * The GEMM accumulates x8 w8 and the LoRA product of T / q_x and
+ * L_A8 = L_A / qw (bf16) in one accumulator and multiplies it by q_x qw[n].
+ * D_in must be a multiple of 256 (whole 256-K stages); D_out a multiple of 8.
+ */
+
+/* Weight preparation, once per layer: W [D_out, D_in] bf16 -> W8 [D_out, D_in]
+ * E4M3 codes (bytes), qw [D_out] float, L_A8 [D_out, R] bf16 = L_A / qw (a
+ * zero qw divides by 1).  L_A and L_A8 may be NULL when R == 0. */
+int rtlynx_quantize_weight_fp8(const void* W, const void* L_A, void* W8, void* qw, void* L_A8, int64_t D_out,
+                               int64_t D_in, int64_t R, void* stream);
+
+/* The FP8 layer, sparse mode: X [M, D_in] bf16, W8 / qw / L_A8 from
+ * rtlynx_quantize_weight_fp8, L_B [R, D_in] bf16, Y [M, D_out] bf16.  Uses
+ * the cached workspace of rtlynx_linear. */
+int rtlynx_linear_fp8(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B, void* Y,
+                      int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* stream);
+
+/* Step 1 of the FP8 form alone, in plain layouts: codes [M, D_in/2] E4M3 of
+ * the kept entries in channel order, meta [M, D_in/4] (one nibble per byte),
+ * qx [M] float.  Any output pointer may be NULL. */
+int rtlynx_sparsify_fp8_debug(const void* X, int64_t M, int64_t D_in, void* codes, void* meta, void* qx,
+                              void* stream);
+
 /* End-to-end form for callers whose activations live in host memory:
  * copies X_host to X_dev, runs rtlynx_linear into Y_dev, copies Y_dev to
  * Y_host.  The work is cut into up to eight token chunks (of at least 512
