@@ -39,7 +39,7 @@ ABI_SYMBOLS = (
     "rtlynx_workspace_layout",
     "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_mlp_block", "rtlynx_linear_noalloc",
     "rtlynx_kernel_launches",
-    "rtlynx_quantize_weight_fp8", "rtlynx_linear_fp8", "rtlynx_sparsify_fp8_debug",
+    "rtlynx_quantize_weight_fp8", "rtlynx_linear_fp8", "rtlynx_linear_fp8_events", "rtlynx_sparsify_fp8_debug",
     "rtlynx_wait_selftest", "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
 )
 
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_quantize_weight_fp8.restype = i
         L.rtlynx_linear_fp8.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p]
         L.rtlynx_linear_fp8.restype = i
+        L.rtlynx_linear_fp8_events.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p]
+        L.rtlynx_linear_fp8_events.restype = i
         L.rtlynx_sparsify_fp8_debug.argtypes = [p, i64, i64, p, p, p, p]
         L.rtlynx_sparsify_fp8_debug.restype = i
         L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
@@ -205,6 +207,16 @@ def rtlynx_quantize_weight_fp8(W, L_A, W8, qw, L_A8, D_out, D_in, R, stream=None
 def rtlynx_linear_fp8(X, W8, qw, L_A8, L_B, Y, M, D_in, D_out, R, stream=None) -> int:
     return _check(lib().rtlynx_linear_fp8(_ptr(X), _ptr(W8), _ptr(qw), _ptr(L_A8), _ptr(L_B), _ptr(Y), M, D_in,
                                           D_out, R, _stream(stream)), "rtlynx_linear_fp8")
+
+
+def rtlynx_linear_fp8_events(X, W8, qw, L_A8, L_B, Y, M, D_in, D_out, R, ev_start, ev_mid, ev_end,
+                             stream=None) -> int:
+    """Events are torch.cuda.Event objects (or raw handles), any may be None."""
+    def h(e):
+        return None if e is None else (e if isinstance(e, int) else int(e.cuda_event))
+    return _check(lib().rtlynx_linear_fp8_events(_ptr(X), _ptr(W8), _ptr(qw), _ptr(L_A8), _ptr(L_B), _ptr(Y), M,
+                                                 D_in, D_out, R, h(ev_start), h(ev_mid), h(ev_end),
+                                                 _stream(stream)), "rtlynx_linear_fp8_events")
 
 
 def rtlynx_sparsify_fp8_debug(X, M, D_in, codes, meta, qx, stream=None) -> int:

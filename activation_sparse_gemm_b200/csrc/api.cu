@@ -515,8 +515,9 @@ int rtlynx_quantize_weight_fp8(const void* W, const void* L_A, void* W8, void* q
                : RTLYNX_OK;
 }
 
-int rtlynx_linear_fp8(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B, void* Y,
-                      int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* stream_) {
+int rtlynx_linear_fp8_events(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B,
+                             void* Y, int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* ev_start,
+                             void* ev_mid, void* ev_end, void* stream_) {
     int rc = validate_fp8(M, D_in, D_out, R);
     if (rc) return rc;
     if (!X || !W8 || !qw || !Y || !aligned16(X) || !aligned16(W8) || !aligned16(qw) || !aligned16(Y))
@@ -536,11 +537,21 @@ int rtlynx_linear_fp8(const void* X, const void* W8, const void* qw, const void*
     if (rc) return rc;
     const Workspace ws = carve(base, l);
     const bool lora = R > 0;
+    auto record = [&](void* ev) {
+        return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev), stream) == cudaSuccess;
+    };
+    if (!record(ev_start)) return RTLYNX_ERR_CUDA;
     if (launch_sparsify(d, X, lora ? L_B : nullptr, ws, di->err_word, stream)) return RTLYNX_ERR_CUDA;
+    if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
     if (launch_gemm(d, true, nullptr, W8, lora ? L_A8 : nullptr, ws, Y, 0, di->num_sms, di->err_word, stream,
                     static_cast<const float*>(qw)))
         return RTLYNX_ERR_CUDA;
-    return RTLYNX_OK;
+    return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+}
+
+int rtlynx_linear_fp8(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B, void* Y,
+                      int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* stream_) {
+    return rtlynx_linear_fp8_events(X, W8, qw, L_A8, L_B, Y, M, D_in, D_out, R, nullptr, nullptr, nullptr, stream_);
 }
 
 int rtlynx_sparsify_fp8_debug(const void* X, int64_t M, int64_t D_in, void* codes, void* meta, void* qx,

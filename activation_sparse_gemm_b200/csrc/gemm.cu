@@ -79,8 +79,9 @@ struct PairShape {
     static constexpr int LORA_A_BYTES = kBM * 64 * 2;
     static constexpr int LORA_B_BYTES = BN_HALF * 64 * 2;
     static constexpr int EPI_BYTES = 4 * 2 * kEpiBufBytes;
+    static constexpr int QW_BYTES = FP8 ? 4 * BN * 4 : 0;  // FP8: each epilogue warp's copy of the tile's q_w
     static constexpr int BAR_BYTES = 1024;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + QW_BYTES + BAR_BYTES + 1024;
     static_assert(BN % (FP8 ? 32 : 16) == 0 && BN >= 64 && 2 * BN + 4 * E_CHUNKS <= 512,
                   "two accumulators (and, when sparse, the metadata) must fit");
     static_assert(B_ATOM_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
@@ -223,7 +224,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi = smem + G::STAGES * G::STAGE_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(epi + G::EPI_BYTES);
+    float* qw_sh = reinterpret_cast<float*>(epi + G::EPI_BYTES);  // FP8 only: [4 warps][BN]
+    uint64_t* full = reinterpret_cast<uint64_t*>(epi + G::EPI_BYTES + G::QW_BYTES);
     uint64_t* empty = full + G::STAGES;
     uint64_t* acc_full = empty + G::STAGES;   // [2]
     uint64_t* acc_empty = acc_full + 2;       // [2], used in the leader only
@@ -434,6 +436,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const int col0 = nt * BN;
             const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN) + lane_addr;
             const bool split = w.unit >= 0;
+            float* qw_w = qw_sh + (warp - 2) * BN;  // FP8: this warp's copy of the tile's q_w
+            if constexpr (FP8) {
+                // one coalesced pass per tile; zero scales (all-zero channels) and
+                // columns past N apply as 1
+                for (int j = lane; j < BN; j += 32) {
+                    const float v = col0 + j < args.N ? args.qw[col0 + j] : 1.0f;
+                    qw_w[j] = v > 0.0f ? v : 1.0f;
+                }
+                __syncwarp();
+            }
             bool write_y = true;
             const int S = args.tail_split;
             const int tt = w.tile - args.full_tiles;  // index among the split tiles
@@ -555,12 +567,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     }
                     if constexpr (FP8) {  // dequantise: q_x of the token times q_w of the column
                         const float qxr = args.qx[row0 + lane];
+                        const float4* w4 = reinterpret_cast<const float4*>(qw_w + c);
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) {
-                            const int col = col0 + c + q;
-                            float w = col < args.N ? args.qw[col] : 1.0f;
-                            w = w > 0.0f ? w : 1.0f;
-                            r[q] = __float_as_uint(__uint_as_float(r[q]) * (qxr * w));
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 w = w4[q];  // the same address in every lane: a broadcast
+                            r[4 * q + 0] = __float_as_uint(__uint_as_float(r[4 * q + 0]) * (qxr * w.x));
+                            r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) * (qxr * w.y));
+                            r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) * (qxr * w.z));
+                            r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) * (qxr * w.w));
                         }
                     }
                     if constexpr (ACT == 1) {

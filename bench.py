@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--workload", default="qkv")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true", help="the layer's FP8 (E4M3) form on the workload's shape")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -449,6 +450,115 @@ def run_block(args):
     return 0
 
 
+def run_fp8(args, wl):
+    """The FP8 (E4M3) form of the layer on a workload's shape: weights prepared
+    once (rtlynx_quantize_weight_fp8, outside the timed region, as a model
+    would at load time), then rtlynx_linear_fp8 per step; one JSON line.  The
+    bf16 sparse layer and cuBLAS's dense FP8 GEMM (torch._scaled_mm, one scale
+    per tensor) on the same shape are timed in the same run."""
+    import numpy as np
+    import torch
+
+    import activation_sparse_gemm_b200 as rl
+    from activation_sparse_gemm_b200.inputs import make_inputs
+
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    rl.lib()
+    X, W, L_A, L_B = make_inputs(wl)
+    M, K, N, R = wl.M, wl.D_in, wl.D_out, wl.R
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+    Xd, Wd, Ad, Bd = dev(X), dev(W), dev(L_A), dev(L_B)
+    W8 = torch.empty((N, K), dtype=torch.uint8, device=device)
+    qw = torch.empty((N,), dtype=torch.float32, device=device)
+    A8 = torch.empty((N, R), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream()
+    rl.rtlynx_quantize_weight_fp8(Wd, Ad, W8, qw, A8, N, K, R, stream)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    def step(e0=None, e1=None, e2=None):
+        rl.rtlynx_linear_fp8_events(Xd, W8, qw, A8, Bd, Y, M, K, N, R, e0, e1, e2, stream)
+
+    def timed(fn, n_events=2):
+        """fn(events) must record the events itself (the library entry points do)."""
+        for _ in range(max(args.warmup, 3)):
+            fn([None] * n_events)
+        evs = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            es = [ev() for _ in range(n_events)]
+            evs.append(es)
+            fn(es)
+        torch.cuda.synchronize()
+        return evs
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    evs = timed(lambda es: step(es[0], None, es[1]))
+    clocks.stop()
+    status = rl.rtlynx_stream_status(stream)
+    if status != rl.OK:
+        raise RuntimeError(f"device-side error: {rl.rtlynx_status_string(status)}")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    pevs = timed(lambda es: step(*es), 3)
+    pro_ms = statistics.mean(a.elapsed_time(b) for a, b, c in pevs)
+    gemm_ms = statistics.mean(b.elapsed_time(c) for a, b, c in pevs)
+    ws_bytes = rl.rtlynx_workspace_size(M, K, N, R, rl.MODE_SPARSE)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    bevs = timed(lambda es: rl.rtlynx_linear_ws_events(Xd, Wd, Ad, Bd, Y, M, K, N, R, rl.MODE_SPARSE, ws, ws_bytes,
+                                                       es[0], None, es[1], stream))
+    bf16_ms = statistics.mean(a.elapsed_time(b) for a, b in bevs)
+    cublas_fp8_us = None
+    try:
+        xa = Xd.to(torch.float8_e4m3fn)
+        wb = Wd.to(torch.float8_e4m3fn)
+        one = torch.ones((), dtype=torch.float32, device=device)
+        for _ in range(max(args.warmup, 3)):
+            torch._scaled_mm(xa, wb.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        cpairs = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            a = ev()
+            torch._scaled_mm(xa, wb.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            cpairs.append((a, ev()))
+        torch.cuda.synchronize()
+        cublas_fp8_us = statistics.mean(a.elapsed_time(b) for a, b in cpairs) * 1e3
+    except Exception as e:  # the baseline is context only
+        cublas_fp8_us = f"unavailable: {type(e).__name__}"
+    flop = wl.dense_equiv_flop
+    gemm_flop = 2 * M * N * K + 2 * M * R * N
+    peaks, peaks_kind = load_peaks()
+    peak = 4.0 * peaks["bf16_tflops"]
+    achieved = gemm_flop / (gemm_ms / 1e3) / 1e12
+    line = {
+        "metric": "fused 2:4 act-sparse+LoRA linear, FP8 (E4M3) operands: us/call, TFLOP/s",
+        "value": flop / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
+        "phases_us": {"sparsify_prologue": pro_ms * 1e3, "sparse_gemm_lora": gemm_ms * 1e3},
+        "bf16_sparse_layer_us": bf16_ms * 1e3, "speedup_vs_bf16_sparse_layer": bf16_ms / ms,
+        "dense_fp8_cublas_us": cublas_fp8_us, "dtype": "e4m3", "vs_baseline": None,
+        "data": "synthetic (seeded, DiT-shaped; random-init weights)",
+        "config": {**workload_desc(wl), "form": "fp8", "l2": "flushed before every timed step (256 MB write)"},
+        "gpu_launches": rl.rtlynx_kernel_launches(M, K, N, R, rl.MODE_SPARSE) * args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "rtlynx_gemm_pair_kernel<sparse, 224, fp8>",
+                     "peak_note": f"4 x {peaks_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s): "
+                                  "fp8 and 2:4 sparse nominal ratios"},
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_lora_fit(args):
     """The closed-form LoRA fit at the qkv shape: 4096 calibration tokens of the
     qkv workload, R = 64; seconds per fit (CUDA events) and the relative error
@@ -521,6 +631,8 @@ def main():
     if args.workload == "lora_fit" and args.impl == "ours":
         return run_lora_fit(args)
     wl = WORKLOADS[args.workload]
+    if args.fp8 and args.impl == "ours":
+        return run_fp8(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

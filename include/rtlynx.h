@@ -135,6 +135,12 @@ int rtlynx_quantize_weight_fp8(const void* W, const void* L_A, void* W8, void* q
 int rtlynx_linear_fp8(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B, void* Y,
                       int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* stream);
 
+/* rtlynx_linear_fp8 that also records caller-created CUDA events (any may
+ * be NULL): before the prologue, between prologue and GEMM, after the GEMM. */
+int rtlynx_linear_fp8_events(const void* X, const void* W8, const void* qw, const void* L_A8, const void* L_B,
+                             void* Y, int64_t M, int64_t D_in, int64_t D_out, int64_t R, void* ev_start,
+                             void* ev_mid, void* ev_end, void* stream);
+
 /* Step 1 of the FP8 form alone, in plain layouts: codes [M, D_in/2] E4M3 of
  * the kept entries in channel order, meta [M, D_in/4] (one nibble per byte),
  * qx [M] float.  Any output pointer may be NULL. */
