@@ -47,6 +47,13 @@
 // 16-column chunk.  Dense-skip tiles: BN = 256, two accumulators filling the
 // 512 columns.
 //
+// FP8 variant (E4M3 operands, tcgen05.mma.sp kind::f8f6f4, K = 64 logical
+// per instruction): BN = 224 (the instruction wants N a multiple of 32); a
+// stage carries 256 logical K in the bf16 stage's A and B bytes plus two
+// metadata chunks, which tcgen05.cp moves into eight tensor-memory columns,
+// two per MMA.  The LoRA stages stay bf16 (T / q_x and L_A / q_w) and add
+// into the same accumulator, and the epilogue multiplies it by q_x q_w.
+//
 // Tensor memory (per CTA, 512 columns): accumulators at [0, BN) and
 // [BN, 2 BN); in sparse mode the metadata of the current 128-wide K chunk at
 // [2 BN, 2 BN + 4).

@@ -22,6 +22,12 @@
 //         s = ||x|| / (||x~|| + 1e-8) in float, and sums the partial T in
 //         segment order, rounded to bf16; then all threads of the CTA rescale
 //         the kept entries in place (s*x rounded once to bf16, nearest even).
+// FP8 mode (the layer's E4M3 form): pass 1 writes the metadata in the 8-bit
+//         operand order (token m of a block at byte 16 m of a chunk, group g
+//         at nibble g) and each segment's max |x| per token; pass 2 forms
+//         q_x = s * max|x| / 448, stores T / q_x, and converts the kept
+//         entries to E4M3 codes of x * (448 / max|x|) in a separate buffer
+//         instead of rescaling them.
 // Both passes and the GEMM launch as programmatic dependents: each one's setup
 // overlaps the previous kernel's tail, and it touches memory only after the
 // grid-dependency wait.
