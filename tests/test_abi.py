@@ -87,3 +87,27 @@ def test_workspace_size_zero_for_dense_and_invalid(lib):
 def test_wait_selftest_rejects_bad_limits_without_launch(lib):
     for limit in (0, -1, 2_000_000_000):
         assert lib.rtlynx_wait_selftest(limit, None) == rl.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M,K,N,R", [
+    (0, 256, 64, 0),      # no tokens
+    (4, 384, 64, 0),      # D_in not a multiple of 256 (whole FP8 stages)
+    (4, 250, 64, 0),
+    (4, 256, 60, 0),      # D_out not a multiple of 8
+    (4, 256, 64, -8),
+])
+def test_fp8_invalid_sizes_rejected_without_launch(lib, M, K, N, R):
+    assert lib.rtlynx_linear_fp8(16, 16, 16, 16, 16, 16, M, K, N, R, None) == rl.ERR_INVALID_ARG
+    if M > 0:  # the weight preparation has no token count
+        assert lib.rtlynx_quantize_weight_fp8(16, 16, 16, 16, 16, N, K, R, None) == rl.ERR_INVALID_ARG
+
+
+def test_fp8_pointers_and_rank_rejected(lib):
+    # null, misaligned, and a LoRA rank without the LoRA factors
+    assert lib.rtlynx_linear_fp8(None, 16, 16, None, None, 16, 4, 256, 64, 0, None) == rl.ERR_INVALID_ARG
+    assert lib.rtlynx_linear_fp8(24, 16, 16, None, None, 16, 4, 256, 64, 0, None) == rl.ERR_INVALID_ARG
+    assert lib.rtlynx_linear_fp8(16, 16, 16, None, None, 16, 4, 256, 64, 64, None) == rl.ERR_INVALID_ARG
+    assert lib.rtlynx_linear_fp8(16, 16, 16, 16, 16, 16, 4, 256, 64, 12, None) == rl.ERR_UNSUPPORTED
+    assert lib.rtlynx_linear_fp8(16, 16, 16, 16, 16, 16, 4, 256, 64, 264, None) == rl.ERR_UNSUPPORTED
+    assert lib.rtlynx_quantize_weight_fp8(16, None, 16, 16, None, 64, 256, 8, None) == rl.ERR_INVALID_ARG
+    assert lib.rtlynx_sparsify_fp8_debug(16, 4, 384, None, None, None, None) == rl.ERR_INVALID_ARG
