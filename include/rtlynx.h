@@ -120,7 +120,12 @@ int rtlynx_sparsify_debug(const void* X, const void* L_B, int64_t M, int64_t D_i
  *   - Y = q_x qw[n] sum(x8 w8) + X L_B^T L_A^T, rounded to bf16.
  * The GEMM accumulates x8 w8 and the LoRA product of T / q_x and
  * L_A8 = L_A / qw (bf16) in one accumulator and multiplies it by q_x qw[n].
- * D_in must be a multiple of 256 (whole 256-K stages); D_out a multiple of 8.
+ * Validation, before anything is launched: a size <= 0, D_in not a multiple
+ * of 256 (whole 256-K stages), D_out not a multiple of 8, a NULL or
+ * misaligned pointer, or R > 0 without the LoRA factors give
+ * RTLYNX_ERR_INVALID_ARG; R not a multiple of 8, or above 256, gives
+ * RTLYNX_ERR_UNSUPPORTED.  Device-side timeouts are reported as for the
+ * bf16 layer (rtlynx_stream_status).
  */
 
 /* Weight preparation, once per layer: W [D_out, D_in] bf16 -> W8 [D_out, D_in]
