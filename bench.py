@@ -462,8 +462,12 @@ def run_fp8(args, wl):
     import activation_sparse_gemm_b200 as rl
     from activation_sparse_gemm_b200.inputs import make_inputs
 
-    torch.cuda.set_device(0)
-    device = torch.device("cuda", 0)
+    from activation_sparse_gemm_b200 import dist as rdist
+    world, rank, local = rdist.env_ranks()
+    if rank != 0:  # a one-GPU measurement: under torchrun only rank 0 runs it
+        return 0
+    torch.cuda.set_device(local if world > 1 else 0)
+    device = torch.device("cuda", torch.cuda.current_device())
     rl.lib()
     X, W, L_A, L_B = make_inputs(wl)
     M, K, N, R = wl.M, wl.D_in, wl.D_out, wl.R
