@@ -38,7 +38,7 @@ ABI_SYMBOLS = (
     "rtlynx_linear", "rtlynx_workspace_size", "rtlynx_linear_ws", "rtlynx_linear_ws_events",
     "rtlynx_workspace_layout",
     "rtlynx_sparsify_debug", "rtlynx_linear_host", "rtlynx_mlp_block", "rtlynx_linear_noalloc",
-    "rtlynx_kernel_launches",
+    "rtlynx_kernel_launches", "rtlynx_schedule_info",
     "rtlynx_quantize_weight_fp8", "rtlynx_linear_fp8", "rtlynx_linear_fp8_events", "rtlynx_sparsify_fp8_debug",
     "rtlynx_wait_selftest", "rtlynx_stream_status", "rtlynx_status_string", "rtlynx_release",
 )
@@ -58,6 +58,12 @@ class WsLayout(ctypes.Structure):
     _fields_ = [("M_pad", ctypes.c_int64), ("Kc_pad", ctypes.c_int64), ("k_chunks", ctypes.c_int64),
                 ("R_pad", ctypes.c_int64), ("vals", ctypes.c_size_t), ("meta", ctypes.c_size_t),
                 ("s", ctypes.c_size_t), ("T", ctypes.c_size_t), ("total", ctypes.c_size_t)]
+
+
+class Schedule(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "prologue_ctas", "prologue_tiles", "prologue_max_segs", "row_blocks", "k_tiles_per_block",
+        "gemm_pairs", "gemm_tiles", "tail_full", "tail_split", "tail_units", "k_stages", "lora_stages")]
 
 
 def lib() -> ctypes.CDLL:
@@ -98,6 +104,8 @@ def lib() -> ctypes.CDLL:
         L.rtlynx_sparsify_fp8_debug.restype = i
         L.rtlynx_kernel_launches.argtypes = [i64, i64, i64, i64, i]
         L.rtlynx_kernel_launches.restype = i
+        L.rtlynx_schedule_info.argtypes = [i64, i64, i64, i64, i, ctypes.POINTER(Schedule)]
+        L.rtlynx_schedule_info.restype = i
         L.rtlynx_wait_selftest.argtypes = [i64, p]
         L.rtlynx_wait_selftest.restype = i
         L.rtlynx_stream_status.argtypes = [p]
@@ -194,7 +202,8 @@ def rtlynx_linear_noalloc(X, W, L_A, L_B, Y, M, D_in, D_out, R, mode, dev_status
     that must not synchronize).  The workspace is a static device array of
     NOALLOC_MAX_BYTES shared by all calls on a device; calls that overlap on the
     GPU race on it.  dev_status: optional device int32 that receives the
-    device-side timeout code."""
+    device-side timeout code; without it a timeout goes to the library's error
+    word, which rtlynx_stream_status reports."""
     return _check(lib().rtlynx_linear_noalloc(_ptr(X), _ptr(W), _ptr(L_A), _ptr(L_B), _ptr(Y), M, D_in, D_out, R,
                                               mode, _ptr(dev_status), _stream(stream)), "rtlynx_linear_noalloc")
 
@@ -226,6 +235,13 @@ def rtlynx_sparsify_fp8_debug(X, M, D_in, codes, meta, qx, stream=None) -> int:
 
 def rtlynx_kernel_launches(M, D_in, D_out, R, mode) -> int:
     return int(lib().rtlynx_kernel_launches(M, D_in, D_out, R, mode))
+
+
+def rtlynx_schedule_info(M, D_in, D_out, R, num_sms) -> Schedule:
+    """The work split of a sparse-mode call on a GPU with num_sms SMs (host only)."""
+    out = Schedule()
+    _check(lib().rtlynx_schedule_info(M, D_in, D_out, R, num_sms, ctypes.byref(out)), "rtlynx_schedule_info")
+    return out
 
 
 def rtlynx_wait_selftest(limit_ns, stream=None) -> int:

@@ -16,8 +16,12 @@ struct DeviceInfo {
     bool init = false;
     bool supported = false;
     int num_sms = 0;
-    int* err_word = nullptr;  // device memory, one int
+    int* err_word = nullptr;  // device address of g_err_word on this device
 };
+
+// The per-device error word: a module variable, so that every device that
+// loads the library has its own copy and no call has to allocate one.
+__device__ int g_err_word;
 
 std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
@@ -57,7 +61,12 @@ int current_device(DeviceInfo** out) {
         di.supported = (major == 10 && minor == 0);
         di.num_sms = sms;
         if (di.supported) {
-            if (cudaMalloc(&di.err_word, sizeof(int)) != cudaSuccess) return RTLYNX_ERR_OOM;
+            void* word = nullptr;
+            if (cudaGetSymbolAddress(&word, g_err_word) != cudaSuccess || word == nullptr) {
+                cudaGetLastError();
+                return RTLYNX_ERR_CUDA;
+            }
+            di.err_word = static_cast<int*>(word);
             if (cudaMemset(di.err_word, 0, sizeof(int)) != cudaSuccess) return RTLYNX_ERR_CUDA;
         }
         if (!g_encode) {
@@ -109,24 +118,49 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// True when the byte ranges [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void* a, uint64_t na, const void* b, uint64_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
 int validate(const void* X, const void* W, const void* L_A, const void* L_B, const void* Y, int64_t M,
              int64_t K, int64_t N, int64_t R, int mode) {
     if (mode != RTLYNX_MODE_SPARSE && mode != RTLYNX_MODE_DENSE_SKIP) return RTLYNX_ERR_INVALID_ARG;
     if (M <= 0 || K <= 0 || N <= 0 || R < 0) return RTLYNX_ERR_INVALID_ARG;
     if (K % 8 != 0 || N % 8 != 0) return RTLYNX_ERR_INVALID_ARG;
-    if (M > (int64_t(1) << 31) - kBM || K > (int64_t(1) << 30) || N > (int64_t(1) << 30))
+    if (M > (int64_t(1) << 31) - 2 * kBM || K > (int64_t(1) << 30) || N > (int64_t(1) << 30))
         return RTLYNX_ERR_UNSUPPORTED;
     if (!X || !W || !Y) return RTLYNX_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(W) || !aligned16(Y)) return RTLYNX_ERR_INVALID_ARG;
-    if (mode == RTLYNX_MODE_SPARSE && R > 0) {
+    const bool lora = mode == RTLYNX_MODE_SPARSE && R > 0;
+    if (lora) {
         if (!L_A || !L_B) return RTLYNX_ERR_INVALID_ARG;
         if (!aligned16(L_A) || !aligned16(L_B)) return RTLYNX_ERR_INVALID_ARG;
         if (R % 8 != 0 || R > 256) return RTLYNX_ERR_UNSUPPORTED;
     }
+    // Y is written while the inputs are still being read: it must not share a
+    // byte with any of them.
+    const uint64_t m = static_cast<uint64_t>(M), k = static_cast<uint64_t>(K), n = static_cast<uint64_t>(N),
+                   r = static_cast<uint64_t>(R);
+    const uint64_t y_bytes = 2 * m * n;
+    if (overlaps(Y, y_bytes, X, 2 * m * k) || overlaps(Y, y_bytes, W, 2 * n * k)) return RTLYNX_ERR_INVALID_ARG;
+    if (lora && (overlaps(Y, y_bytes, L_A, 2 * n * r) || overlaps(Y, y_bytes, L_B, 2 * r * k)))
+        return RTLYNX_ERR_INVALID_ARG;
     return RTLYNX_OK;
 }
 
-}  // namespace
+int device_info(int* num_sms, int** err_word) {
+    DeviceInfo* di = nullptr;
+    const int rc = current_device(&di);
+    if (rc) return rc;
+    *num_sms = di->num_sms;
+    *err_word = di->err_word;
+    return RTLYNX_OK;
+}
 
 bool ensure_tmap_encoder() {
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -234,7 +268,7 @@ Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms, bool fp8
     const int64_t max_pairs = (num_sms > 0 ? num_sms : 148) / 2;
     d.gemm_pairs = d.gemm_tiles < max_pairs ? d.gemm_tiles : max_pairs;
     const int64_t rem = d.gemm_tiles % d.gemm_pairs;
-    const int64_t n_iter = (fp8 ? d.k_chunks / 2 : d.k_chunks) + d.R_pad / 64;
+    const int64_t n_iter = sparse_k_stages(d) + sparse_lora_stages(d);
     int64_t split = rem > 0 ? d.gemm_pairs / rem : 1;
     if (split > kMaxSplit) split = kMaxSplit;
     if (split > n_iter / 2) split = n_iter / 2;
@@ -523,7 +557,14 @@ int rtlynx_linear_fp8_events(const void* X, const void* W8, const void* qw, cons
     if (!X || !W8 || !qw || !Y || !aligned16(X) || !aligned16(W8) || !aligned16(qw) || !aligned16(Y))
         return RTLYNX_ERR_INVALID_ARG;
     if (R > 0 && (!L_A8 || !L_B || !aligned16(L_A8) || !aligned16(L_B))) return RTLYNX_ERR_INVALID_ARG;
-    if (Y == X) return RTLYNX_ERR_INVALID_ARG;
+    {
+        const uint64_t m = static_cast<uint64_t>(M), k = static_cast<uint64_t>(D_in), n = static_cast<uint64_t>(D_out),
+                       r = static_cast<uint64_t>(R);
+        const uint64_t yb = 2 * m * n;
+        if (overlaps(Y, yb, X, 2 * m * k) || overlaps(Y, yb, W8, n * k) || overlaps(Y, yb, qw, 4 * n) ||
+            (R > 0 && (overlaps(Y, yb, L_A8, 2 * n * r) || overlaps(Y, yb, L_B, 2 * r * k))))
+            return RTLYNX_ERR_INVALID_ARG;
+    }
     DeviceInfo* di = nullptr;
     rc = current_device(&di);
     if (rc) return rc;
@@ -639,6 +680,28 @@ int rtlynx_linear_host(const void* X_host, const void* W, const void* L_A, const
     return rc;
 }
 
+int rtlynx_schedule_info(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int num_sms, rtlynx_schedule* out) {
+    if (!out || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8 || num_sms < 2 ||
+        num_sms > 1024)
+        return RTLYNX_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31) - 2 * kBM || D_in > (int64_t(1) << 30) || D_out > (int64_t(1) << 30))
+        return RTLYNX_ERR_UNSUPPORTED;
+    const Dims d = make_dims(M, D_in, D_out, R, num_sms);
+    out->prologue_ctas = d.grid1;
+    out->prologue_tiles = d.m_blocks * d.kt2;
+    out->prologue_max_segs = d.max_segs;
+    out->row_blocks = d.m_blocks;
+    out->k_tiles_per_block = d.kt2;
+    out->gemm_pairs = d.gemm_pairs;
+    out->gemm_tiles = d.gemm_tiles;
+    out->tail_full = d.tail_full;
+    out->tail_split = d.tail_split;
+    out->tail_units = d.tail_units;
+    out->k_stages = sparse_k_stages(d);
+    out->lora_stages = sparse_lora_stages(d);
+    return RTLYNX_OK;
+}
+
 int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode) {
     if (mode == RTLYNX_MODE_DENSE_SKIP) return (M > 0 && D_in > 0 && D_out > 0) ? 1 : 0;
     if (mode != RTLYNX_MODE_SPARSE || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8) return 0;
@@ -713,13 +776,8 @@ void rtlynx_release(void) {
             hp = HostPipe{};
         }
     }
-    for (int i = 0; i < kMaxDevices; ++i) {
-        if (g_dev[i].err_word) {
-            cudaSetDevice(i);
-            cudaFree(g_dev[i].err_word);
-        }
-        g_dev[i] = DeviceInfo{};
-    }
+    // the error words are module variables: nothing to free
+    for (int i = 0; i < kMaxDevices; ++i) g_dev[i] = DeviceInfo{};
     cudaSetDevice(cur);
 }
 

@@ -732,8 +732,8 @@ int launch_gemm(const Dims& d, bool sparse, const void* A, const void* W, const 
     args.N = static_cast<int>(d.N);
     args.m_pairs = static_cast<int>((d.M + 2 * kBM - 1) / (2 * kBM));
     args.n_tiles = static_cast<int>((d.N + BN - 1) / BN);
-    args.k_stages = static_cast<int>(fp8 ? d.k_chunks / 2 : (sparse ? d.k_chunks : d.k_tiles));
-    args.lora_stages = lora ? static_cast<int>(d.R_pad / 64) : 0;
+    args.k_stages = static_cast<int>(sparse ? sparse_k_stages(d) : d.k_tiles);
+    args.lora_stages = lora ? static_cast<int>(sparse_lora_stages(d)) : 0;
     args.k_chunks = static_cast<int>(d.k_chunks);
     {
         // While both operands fit in L2 (126 MB) the row-pair-fastest order

@@ -61,6 +61,12 @@ struct WsLayout {
     size_t total;
 };
 
+// Main-loop and LoRA stages of one sparse GEMM tile (the split of the last
+// wave and the kernel's schedule use the same counts): a bf16 stage covers
+// one 128-wide metadata chunk, an FP8 stage two; a LoRA-up stage 64 of R.
+inline int64_t sparse_k_stages(const Dims& d) { return d.fp8 ? d.k_chunks / 2 : d.k_chunks; }
+inline int64_t sparse_lora_stages(const Dims& d) { return d.R_pad / 64; }
+
 Dims make_dims(int64_t M, int64_t K, int64_t N, int64_t R, int num_sms, bool fp8 = false);
 WsLayout make_ws_layout(const Dims& d);
 
@@ -140,6 +146,13 @@ int launch_quantize_weight_fp8(const void* W, const void* L_A, void* W8, float* 
 int launch_unpack_fp8_debug(const Dims& d, const Workspace& ws, void* codes, void* meta, void* qx,
                             cudaStream_t stream);
 // Shared by the entry points (api.cu).
+// Argument checks of one layer call; returns an rtlynx_status (nothing is
+// launched).  Y must not share a byte with X, W, L_A or L_B.
+int validate(const void* X, const void* W, const void* L_A, const void* L_B, const void* Y, int64_t M,
+             int64_t K, int64_t N, int64_t R, int mode);
+// The current device's SM count and the device address of the library's
+// error word on it; an rtlynx_status.  Allocates nothing.
+int device_info(int* num_sms, int** err_word);
 bool ensure_tmap_encoder();
 Workspace carve(void* base, const WsLayout& l);
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,

@@ -17,8 +17,9 @@
  *       X [M, D_in], W [D_out, D_in] (nn.Linear layout), L_A [D_out, R],
  *       L_B [R, D_in], Y [M, D_out].
  *   - Pointers are device memory owned by the caller unless a name ends in
- *     _host.  Inputs are only read.  Y is overwritten; it must not overlap
- *     an input.  Every pointer must be 16-byte aligned.
+ *     _host.  Inputs are only read.  Y is overwritten; a Y that shares a byte
+ *     with an input is rejected with RTLYNX_ERR_INVALID_ARG.  Every pointer
+ *     must be 16-byte aligned.
  *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls are asynchronous on that stream; nothing synchronizes the host
  *     unless stated.
@@ -71,8 +72,8 @@ int rtlynx_linear(const void* X, const void* W, const void* L_A, const void* L_B
 size_t rtlynx_workspace_size(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode);
 
 /* rtlynx_linear with a caller-owned device workspace of ws_bytes bytes
- * (>= rtlynx_workspace_size, 256-byte aligned).  Allocates nothing except,
- * on a device's first call, its 4-byte device error word. */
+ * (>= rtlynx_workspace_size, 256-byte aligned).  Allocates nothing (the
+ * device error word is a module variable of the library). */
 int rtlynx_linear_ws(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
                      int64_t D_in, int64_t D_out, int64_t R, int mode, void* workspace, size_t ws_bytes,
                      void* stream);
@@ -211,10 +212,14 @@ int rtlynx_mlp_block(const void* X, const void* W_up, const void* LA_up, const v
  * entry point holds until the process exits; problems whose workspace
  * (rtlynx_workspace_size) is larger are rejected with RTLYNX_ERR_UNSUPPORTED
  * before anything is launched.
- *   dev_status  a caller-owned, 4-byte-aligned device int (or NULL): a
- *               bounded device-side wait that runs out stores
- *               RTLYNX_ERR_DEVICE_TIMEOUT's device code (1) there; the caller
- *               zeroes it beforehand and reads it after synchronizing.
+ *   dev_status  a caller-owned, 4-byte-aligned device int, or NULL.  A
+ *               bounded device-side wait that runs out stores a nonzero code
+ *               (1) there, the kernels of the call then stop early, and Y is
+ *               incomplete; the caller zeroes the int beforehand and reads it
+ *               after synchronizing.  With NULL the code goes to the library's
+ *               own per-device error word (a module variable, no allocation),
+ *               which rtlynx_stream_status reports as RTLYNX_ERR_DEVICE_TIMEOUT
+ *               and clears, exactly as for rtlynx_linear.
  * Other arguments as rtlynx_linear.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) and reads device properties;
  * make it outside any stream capture.  Every call shares the one array and
@@ -224,6 +229,27 @@ int rtlynx_mlp_block(const void* X, const void* W_up, const void* LA_up, const v
  */
 int rtlynx_linear_noalloc(const void* X, const void* W, const void* L_A, const void* L_B, void* Y, int64_t M,
                           int64_t D_in, int64_t D_out, int64_t R, int mode, int* dev_status, void* stream);
+
+/* The work split one sparse-mode call uses on a GPU with num_sms SMs (2 ..
+ * 1024), computed on the host alone (no GPU needed):
+ *   prologue_ctas      CTAs of the streaming sparsify pass; CTA c takes the
+ *                      tiles [c T / G, (c + 1) T / G) of the T = prologue_tiles
+ *                      (row block x 64-wide K tile) tiles, G = prologue_ctas,
+ *                      row block b owning tiles [b k, (b + 1) k), k =
+ *                      k_tiles_per_block
+ *   prologue_max_segs  the most CTAs whose tiles meet one row block (the
+ *                      partial-sum slots the workspace holds per token)
+ *   gemm_pairs, gemm_tiles  persistent CTA pairs and 256 x 240 output tiles
+ *   tail_full, tail_split, tail_units  tiles [0, tail_full) run whole; each
+ *                      later tile is cut along its stages into tail_split
+ *                      parts (tail_units parts in all, one per pair)
+ *   k_stages, lora_stages  pipeline stages of one tile (main loop, LoRA-up)
+ * RTLYNX_ERR_INVALID_ARG for invalid sizes or a NULL out. */
+typedef struct {
+    int64_t prologue_ctas, prologue_tiles, prologue_max_segs, row_blocks, k_tiles_per_block;
+    int64_t gemm_pairs, gemm_tiles, tail_full, tail_split, tail_units, k_stages, lora_stages;
+} rtlynx_schedule;
+int rtlynx_schedule_info(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int num_sms, rtlynx_schedule* out);
 
 /* Number of kernels one rtlynx_linear call with these sizes launches (0 for
  * invalid sizes): the sparse path launches its prologue kernel(s) and the GEMM,

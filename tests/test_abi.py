@@ -69,8 +69,43 @@ def test_null_and_misaligned_pointers_rejected(lib):
 
 
 def test_unsupported_rank_rejected(lib):
-    assert lib.rtlynx_linear(16, 16, 16, 16, 16, 4, 64, 64, 264, 0, None) == rl.ERR_UNSUPPORTED
-    assert lib.rtlynx_linear(16, 16, 16, 16, 16, 4, 64, 64, 12, 0, None) == rl.ERR_UNSUPPORTED
+    X, W, A, B, Y = 1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20  # distinct, far apart
+    assert lib.rtlynx_linear(X, W, A, B, Y, 4, 64, 64, 264, 0, None) == rl.ERR_UNSUPPORTED
+    assert lib.rtlynx_linear(X, W, A, B, Y, 4, 64, 64, 12, 0, None) == rl.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("entry", ["linear", "ws", "noalloc", "host"])
+def test_output_overlapping_an_input_rejected(lib, entry):
+    """Y sharing a byte with X, W, L_A or L_B is rejected before anything runs
+    (the pointers are never dereferenced, so fake addresses do)."""
+    M, K, N, R = 4, 64, 32, 16
+    base = {"X": 1 << 20, "W": 2 << 20, "L_A": 3 << 20, "L_B": 4 << 20}
+    sizes = {"X": 2 * M * K, "W": 2 * N * K, "L_A": 2 * N * R, "L_B": 2 * R * K}
+
+    def call(Y, args):
+        if entry == "linear":
+            return lib.rtlynx_linear(args["X"], args["W"], args["L_A"], args["L_B"], Y, M, K, N, R, 0, None)
+        if entry == "ws":
+            return lib.rtlynx_linear_ws(args["X"], args["W"], args["L_A"], args["L_B"], Y, M, K, N, R, 0, 1 << 30,
+                                        1 << 20, None)
+        if entry == "noalloc":
+            return lib.rtlynx_linear_noalloc(args["X"], args["W"], args["L_A"], args["L_B"], Y, M, K, N, R, 0, None,
+                                             None)
+        return lib.rtlynx_linear_host(1 << 31, args["W"], args["L_A"], args["L_B"], 3 << 30, M, K, N, R, 0,
+                                      args["X"], Y, None)
+
+    for name, addr in base.items():
+        # Y's last 16 bytes on the input's first 16, and Y starting on the input's last 16
+        y_bytes = 2 * M * N
+        for Y in (addr - y_bytes + 16, addr + sizes[name] - 16):
+            assert call(Y, base) == rl.ERR_INVALID_ARG, (entry, name, Y)
+
+
+def test_fp8_output_overlapping_an_input_rejected(lib):
+    M, K, N, R = 4, 256, 32, 16
+    X, W8, qw, A8, B = 1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20
+    for Y in (X + 2 * M * K - 16, W8 + N * K - 16, qw, A8 + 16, B):
+        assert lib.rtlynx_linear_fp8(X, W8, qw, A8, B, Y, M, K, N, R, None) == rl.ERR_INVALID_ARG
 
 
 def test_python_binding_raises_on_error(lib):

@@ -57,6 +57,42 @@ def test_noalloc_matches_linear_on_consecutive_calls():
         assert np.isfinite(bf16_bits_to_f32(got)).all()
 
 
+def test_noalloc_split_tail_tickets_reused():
+    """Shapes whose GEMM cuts its last tiles along K, so that the fp32 partials
+    and the arrival tickets of the split tiles live in the shared static array:
+    two different split shapes back to back, then the first again, each equal
+    bit for bit to rtlynx_linear (which uses its own workspace)."""
+    import torch
+    shapes = [(2560, 1024, 2160, 64), (2560, 2048, 1920, 64), (2560, 1024, 2160, 64)]
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        for M, K, N, R in shapes[:2]:
+            s = rl.rtlynx_schedule_info(M, K, N, R, 148)
+            assert s.tail_units > 0, (M, K, N)  # the shape really splits
+    for M, K, N, R in shapes:
+        assert rl.rtlynx_workspace_size(M, K, N, R, rl.MODE_SPARSE) <= rl.NOALLOC_MAX_BYTES
+        X, W, L_A, L_B = make_custom(M, K, N, R, seed=60 + K + N)
+        ref, got, status = _both(X, W, L_A, L_B, rl.MODE_SPARSE)
+        assert status == 0
+        assert np.array_equal(ref, got), f"noalloc output differs from rtlynx_linear at {M}x{K}x{N}"
+
+
+def test_noalloc_without_status_word():
+    """With no caller status word, a timeout would go to the library's own
+    error word: the call still allocates nothing, its output equals
+    rtlynx_linear's, and rtlynx_stream_status reports OK."""
+    import torch
+    X, W, L_A, L_B = make_custom(300, 512, 264, 32, seed=43)
+    M, K = X.shape
+    N, R = W.shape[0], L_B.shape[0]
+    Xd, Wd, Ad, Bd = _dev(X), _dev(W), _dev(L_A), _dev(L_B)
+    Y_ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Y_na = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rl.rtlynx_linear(Xd, Wd, Ad, Bd, Y_ref, M, K, N, R, rl.MODE_SPARSE)
+    rl.rtlynx_linear_noalloc(Xd, Wd, Ad, Bd, Y_na, M, K, N, R, rl.MODE_SPARSE, None)
+    assert rl.rtlynx_stream_status() == rl.OK
+    assert np.array_equal(_bits(Y_ref), _bits(Y_na))
+
+
 def test_noalloc_dense_skip_and_no_lora():
     X, W, L_A, L_B = make_custom(129, 256, 136, 16, seed=42)
     for mode, la, lb in ((rl.MODE_DENSE_SKIP, None, None), (rl.MODE_SPARSE, None, None)):
