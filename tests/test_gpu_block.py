@@ -23,7 +23,9 @@ pipeline paragraph).  Bars:
         most tokens hold a flip somewhere;
       * all tokens together: relative Frobenius error <= 2e-2.
     The down-projection alone meets the full bar on the oracle's own inputs
-    (the mlp_down cases of test_gpu_parity.py).
+    (the mlp_down cases of test_gpu_parity.py), and the block's Y meets it
+    against the oracle's down-projection of the kernel's own H (the strong
+    check in check_block).
 """
 import numpy as np
 import pytest
@@ -32,7 +34,7 @@ import oracle
 import activation_sparse_gemm_b200 as rl
 from activation_sparse_gemm_b200.inputs import bf16_bits_to_f32, make_block_inputs
 
-from tests.test_gpu_parity import dev, host_bits, run_sparsify
+from tests.test_gpu_parity import assert_y_close, dev, host_bits, run_sparsify
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +64,14 @@ def run_block(args, mode_up, mode_down):
 
 def check_block(args, mode_up, mode_down, rows=None):
     H, Y = run_block(args, mode_up, mode_down)
+    # The strong check: the block's Y is the down-projection layer applied to
+    # the H the block produced, against the oracle run on that same H, at the
+    # single-layer bar.
+    X, W_up, LA_up, LB_up, W_down, LA_down, LB_down = args
+    sparse_down = mode_down == rl.MODE_SPARSE
+    Y_on_H = oracle.linear(H, W_down, LA_down if sparse_down else None, LB_down if sparse_down else None,
+                           mode=mode_down, rows=rows)
+    assert_y_close(Y if rows is None else Y[rows], Y_on_H, "block Y against the oracle on the kernel's H")
     Y_up_ref, H_ref, Y_ref = oracle.mlp_block(*args, mode_up=mode_up, mode_down=mode_down, rows=rows)
     if rows is not None:
         H, Y = H[rows], Y[rows]

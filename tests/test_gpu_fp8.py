@@ -34,6 +34,15 @@ def quantize_weight(W, L_A):
     return W8, qw, L_A8
 
 
+def oracle_weights(W, W8_gpu, qw_gpu):
+    """The oracle's quantised weights, asserted equal to the GPU's: every Y
+    reference below is built from these, never from the GPU's."""
+    rW8, rqw = oracle.quantize_weight_fp8(W)
+    assert (W8_gpu == rW8).all(), "W8 codes differ from the oracle's"
+    assert (qw_gpu == rqw).all(), "qw differs from the oracle's"
+    return rW8, rqw
+
+
 def run_fp8(X, W, L_A, L_B):
     import torch
     M, K = X.shape
@@ -89,18 +98,22 @@ def test_fp8_linear_small(M, K, N, R):
     if R == 0:
         L_A = L_B = None
     Y, W8, qw, _ = run_fp8(X, W, L_A, L_B)
-    Y_ref = oracle.linear_fp8(X, W8, qw, L_A, L_B)
-    assert_y_close(Y, Y_ref, f"fp8 {M}x{K}x{N} R={R}", edge=True)
+    rW8, rqw = oracle_weights(W, W8, qw)
+    Y_ref = oracle.linear_fp8(X, rW8, rqw, L_A, L_B)
+    assert_y_close(Y, Y_ref, f"fp8 {M}x{K}x{N} R={R}")
 
 
 def test_fp8_qkv_shape_sampled():
-    """The qkv workload's shape (4096 x 3072 -> 9216, R = 64), sampled tokens."""
+    """The qkv workload's shape (4096 x 3072 -> 9216, R = 64): the GPU's weight
+    codes and scales equal the oracle's on the whole W; Y on a whole 256-row
+    band and 65 further tokens, against the oracle on the oracle's codes."""
     wl = WORKLOADS["qkv"]
     X, W, L_A, L_B = make_inputs(wl)
     Y, W8, qw, _ = run_fp8(X, W, L_A, L_B)
+    rW8, rqw = oracle_weights(W, W8, qw)
     rng = np.random.default_rng(4)
-    rows = sorted(set([0, 127, 128, 255, 4095] + rng.integers(0, wl.M, 11).tolist()))
-    Y_ref = oracle.linear_fp8(X, W8, qw, L_A, L_B, rows=rows)
+    rows = sorted(set(list(range(0, 256)) + [4095] + rng.integers(0, wl.M, 64).tolist()))
+    Y_ref = oracle.linear_fp8(X, rW8, rqw, L_A, L_B, rows=rows)
     assert_y_close(Y[rows], Y_ref, "fp8 qkv")
     # FP8 against the bf16 layer: the quantisation error itself, for the record
     Y16 = oracle.linear(X, W, L_A, L_B, rows=rows)

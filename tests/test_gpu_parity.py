@@ -34,10 +34,24 @@ def f64(bits):
     return bf16_bits_to_f32(bits).astype(np.float64)
 
 
-def assert_y_close(Y_gpu_bits, Y_ref, what="", edge=False):
-    """The stated bar on Y.  For edge shapes (tiny K, ragged tails) whose
-    output has entries far above its RMS, the bf16 rounding of Y itself can
-    reach 2^-9 |Y|; there the element bar also admits 2^-8 |Y_ref|."""
+def bf16_bracket(y):
+    """The two bf16 values enclosing each exact (float64) value: lo <= y <= hi,
+    equal when y is representable (normal range)."""
+    y = np.asarray(y, np.float64)
+    _, p = np.frexp(y)                 # |y| = m 2^p, 0.5 <= m < 1
+    ulp = np.ldexp(1.0, p - 8)         # 8 significant bits
+    lo = np.floor(y / ulp) * ulp
+    hi = np.ceil(y / ulp) * ulp
+    return lo, hi
+
+
+def assert_y_close(Y_gpu_bits, Y_ref, what=""):
+    """The stated bar on Y: ||Y - Y_ref||_F <= 5e-3 ||Y_ref||_F, and per element
+    |Y - Y_ref| <= 2e-2 RMS(Y_ref).  The element bar is finer than bf16's own
+    spacing once |Y_ref| > 2^8 * 2e-2 RMS (about 5 RMS): there no bf16 output,
+    the correctly rounded exact value included, can meet it.  An element above
+    the bar therefore passes only if it is one of the two bf16 values that
+    enclose the exact result (the best a bf16 output can hold)."""
     Y = f64(Y_gpu_bits)
     err = Y - Y_ref
     ref_norm = np.linalg.norm(Y_ref)
@@ -45,10 +59,17 @@ def assert_y_close(Y_gpu_bits, Y_ref, what="", edge=False):
     rel = np.linalg.norm(err) / ref_norm if ref_norm > 0 else np.linalg.norm(err)
     assert np.isfinite(Y).all(), what
     assert rel <= REL_FRO, f"{what}: rel Frobenius error {rel:.3e}"
-    bound = MAX_RMS * rms + (2.0 ** -8 * np.abs(Y_ref) if edge else 0.0) + 1e-30
-    worst = np.argmax(np.abs(err) - bound)
-    assert (np.abs(err) <= bound).all(), \
-        f"{what}: error {np.abs(err).flat[worst]:.3e} at |Y_ref| {np.abs(Y_ref).flat[worst]:.3e}, RMS {rms:.3e}"
+    bound = MAX_RMS * rms + 1e-30
+    over = np.abs(err) > bound
+    if over.any():
+        lo, hi = bf16_bracket(Y_ref[over])
+        enclosing = (Y[over] == lo) | (Y[over] == hi)
+        idx = np.flatnonzero(over)[~enclosing]
+        assert enclosing.all(), \
+            f"{what}: error {np.abs(err).flat[idx[0]]:.3e} at |Y_ref| {np.abs(Y_ref).flat[idx[0]]:.3e}, RMS {rms:.3e}" \
+            f" ({idx.size} outputs above the bar and not a bf16 neighbour of the exact value)"
+        # where the bar binds, it binds only through bf16's spacing
+        assert (np.abs(Y_ref[over]) > 2.0 ** 8 * MAX_RMS * rms * 0.5).all(), f"{what}: bracket rule used below 2.5 RMS"
 
 
 def run_linear(X, W, L_A, L_B, mode=rl.MODE_SPARSE):
@@ -97,7 +118,7 @@ def bf16_ulp_dist(a, b):
     return np.abs(ia - ib)
 
 
-def check_sparsify(X, L_B, rows=None):
+def check_sparsify(X, L_B, rows=None, return_outputs=False):
     vals, meta, s, T = run_sparsify(X, L_B)
     Xs = X if rows is None else X[rows]
     if rows is not None:
@@ -114,8 +135,12 @@ def check_sparsify(X, L_B, rows=None):
         R = L_B.shape[0]
         _, Tref = oracle.linear(Xs, np.zeros((8, K), np.uint16), np.zeros((8, R), np.uint16), L_B, want_T=True)
         err = np.abs(f64(T) - Tref)
-        scale = np.abs(f64(Xs)) @ np.abs(f64(L_B)).T  # sum |x| |l| per entry
-        assert (err <= 2.0 ** -8 * np.abs(Tref) + 2e-5 * scale + 1e-30).all(), "T out of tolerance"
+        # sum |x| |l| per entry (a tolerance term: float32 is ample)
+        scale = np.abs(bf16_bits_to_f32(Xs)) @ np.abs(bf16_bits_to_f32(L_B)).T
+        assert (err <= 2.0 ** -8 * np.abs(Tref) + 2e-5 * scale.astype(np.float64) + 1e-30).all(), \
+            "T out of tolerance"
+    if return_outputs:
+        return same.mean(), meta, s
     return same.mean()
 
 
@@ -124,7 +149,7 @@ def check_sparsify(X, L_B, rows=None):
 def test_dense_skip_small(M, K, N):
     X, W, _, _ = make_custom(M, K, N, 8, seed=100 + M)
     Y = run_linear(X, W, None, None, mode=rl.MODE_DENSE_SKIP)
-    assert_y_close(Y, oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP), "dense-skip", edge=True)
+    assert_y_close(Y, oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP), "dense-skip")
 
 
 # ------------------------------------------------------------------ sparsify prologue
@@ -185,7 +210,7 @@ def test_sparse_linear_small(M, K, N, R):
     if R == 0:
         L_A = L_B = None
     Y = run_linear(X, W, L_A, L_B)
-    assert_y_close(Y, oracle.linear(X, W, L_A, L_B), f"sparse {M}x{K}x{N} R={R}", edge=True)
+    assert_y_close(Y, oracle.linear(X, W, L_A, L_B), f"sparse {M}x{K}x{N} R={R}")
 
 
 def test_tiny_workload_full_parity():
@@ -231,9 +256,7 @@ def test_split_tail_tiles(M, K, N, R):
     X, W, L_A, L_B = make_custom(M, K, N, R, seed=500 + K)
     Y = run_linear(X, W, L_A, L_B)
     Y_ref = oracle.linear(X, W, L_A, L_B)
-    # Outputs several times the RMS occur at this size; their bf16 rounding
-    # alone can exceed 2e-2 RMS, hence the rounding allowance (edge=True).
-    assert_y_close(Y, Y_ref, f"split tail {M}x{K}x{N} R={R}", edge=True)
+    assert_y_close(Y, Y_ref, f"split tail {M}x{K}x{N} R={R}")
     # the split tiles are tiles 74..79 of the raster; operands this small fit
     # in L2, so the raster is row pair fastest (column-tile groups of width 1)
     m_pairs, n_tiles = M // 256, (N + 239) // 240
@@ -250,28 +273,44 @@ def test_split_tail_tiles(M, K, N, R):
     assert (run_linear(X, W, L_A, L_B) == Y).all()
 
 
-# ------------------------------------------------------------------ full-size workloads, sampled
-@pytest.mark.parametrize("name", ["qkv", "mlp_up", "mlp_down", "video"])
-def test_full_workload_sampled(name):
+# ------------------------------------------------------------------ full-size workloads, every token
+@pytest.mark.parametrize("name", ["tiny", "qkv", "mlp_up", "mlp_down", "video"])
+def test_full_workload_prologue_every_token(name):
+    """Metadata bit-exact, values within 1 bf16 ulp (identical where s is), s
+    within 2 float32 ulp and T within its bar, on every token of the workload,
+    at its full size and in the launch configuration the bench times."""
     wl = WORKLOADS[name]
     X, W, L_A, L_B = make_inputs(wl)
-    rng = np.random.default_rng(wl.seed)
-    rows = sorted(set([0, 1, 127, 128, wl.M // 2, wl.M - 1] + rng.integers(0, wl.M, 10).tolist()))
-    Y = run_linear(X, W, L_A, L_B)
-    assert_y_close(Y[rows], oracle.linear(X, W, L_A, L_B, rows=rows), name)
-    vals, meta, s, T = run_sparsify(X, L_B)
-    rmeta, rvals, rs = oracle.sparsify(X[rows])
-    assert (meta[rows] == rmeta).all()
-    assert (ulp_dist_f32(s[rows], rs) <= 2).all()
-    assert (bf16_ulp_dist(vals[rows], rvals) <= 1).all()
-    # properties at any size: metadata is a valid 2:4 pattern everywhere
+    frac_same, meta, s = check_sparsify(X, L_B, return_outputs=True)
+    assert frac_same > 0.99
     assert set(np.unique(meta).tolist()) <= {0x4, 0x8, 0xC, 0x9, 0xD, 0xE}
-    s_all = s
     nz = np.abs(f64(X)).sum(axis=1) > 0
-    assert (s_all[nz] >= 1.0).all() and (s_all[nz] <= np.float32(np.sqrt(2.0)) * np.float32(1 + 2 ** -23)).all()
-    if name == "mlp_down":
-        Yd = run_linear(X, W, None, None, mode=rl.MODE_DENSE_SKIP)
-        assert_y_close(Yd[rows], oracle.linear(X, W, mode=oracle.MODE_DENSE_SKIP, rows=rows), "mlp_down dense")
+    assert (s[nz] >= 1.0).all() and (s[nz] <= np.float32(np.sqrt(2.0)) * np.float32(1 + 2 ** -23)).all()
+
+
+def _video_rows(M):
+    # every token of the first, a middle and the last 256-row band (the last
+    # holds the 120-row tail of M = 32760), and one token in 64 elsewhere
+    mid = (M // 2) // 256 * 256
+    last = (M - 1) // 256 * 256
+    rows = set(range(0, 256)) | set(range(mid, mid + 256)) | set(range(last, M)) | set(range(0, M, 64))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name,mode", [("qkv", rl.MODE_SPARSE), ("mlp_up", rl.MODE_SPARSE),
+                                       ("mlp_down", rl.MODE_SPARSE), ("mlp_down", rl.MODE_DENSE_SKIP),
+                                       ("video", rl.MODE_SPARSE)])
+def test_full_workload_y(name, mode):
+    """Y against the oracle at the plain stated bar (no rounding allowance):
+    every token of qkv, mlp_up and mlp_down (both modes); the video workload
+    on three whole 256-row bands and one token in 64."""
+    wl = WORKLOADS[name]
+    X, W, L_A, L_B = make_inputs(wl)
+    dense = mode == rl.MODE_DENSE_SKIP
+    Y = run_linear(X, W, None if dense else L_A, None if dense else L_B, mode=mode)
+    rows = _video_rows(wl.M) if name == "video" else None
+    ref = oracle.linear(X, W, None if dense else L_A, None if dense else L_B, mode=mode, rows=rows)
+    assert_y_close(Y if rows is None else Y[rows], ref, f"{name} mode={mode}")
 
 
 # ------------------------------------------------------------------ workspace and stream contracts
@@ -320,7 +359,7 @@ def test_two_streams_at_once():
                 outs.append(Y)
         torch.cuda.synchronize()
     for (X, W, L_A, L_B), Y in zip(probs, outs):
-        assert_y_close(host_bits(Y), oracle.linear(X, W, L_A, L_B), "two streams", edge=True)
+        assert_y_close(host_bits(Y), oracle.linear(X, W, L_A, L_B), "two streams")
     assert rl.rtlynx_stream_status(streams[0]) == rl.OK and rl.rtlynx_stream_status(streams[1]) == rl.OK
 
 
@@ -349,7 +388,7 @@ def test_linear_host_buffers_pipelined(M, K, N, R, mode):
     s.synchronize()
     Y = Yh.view(torch.int16).numpy().view(np.uint16)
     ref = oracle.linear(X, W, L_A if lora else None, L_B if lora else None, mode=mode)
-    assert_y_close(Y, ref, f"host {M}x{K}x{N}", edge=True)
+    assert_y_close(Y, ref, f"host {M}x{K}x{N}")
     assert (host_bits(Ycopy) == Y).all()
     assert (host_bits(Xd) == X).all()
 
@@ -364,5 +403,5 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert rl.rtlynx_stream_status() == rl.OK  # the status word was cleared
     X, W, L_A, L_B = make_custom(130, 256, 128, 32, seed=77)
     Y = run_linear(X, W, L_A, L_B)
-    assert_y_close(Y, oracle.linear(X, W, L_A, L_B), "after timeout", edge=True)
+    assert_y_close(Y, oracle.linear(X, W, L_A, L_B), "after timeout")
     torch.cuda.synchronize()
