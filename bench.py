@@ -1,6 +1,6 @@
 """Benchmark of the RT-Lynx fused activation-sparse + LoRA linear layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qkv] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload video] [--impl ours|reference]
     python bench.py --workload dit_mlp   (the feed-forward block of two layers, one GPU)
     python bench.py --workload lora_fit  (the closed-form LoRA fit and the error it removes, one GPU)
 
@@ -39,7 +39,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qkv")
+    # the headline: the largest single-GPU configuration (32760 tokens, 5120 -> 13824)
+    ap.add_argument("--workload", default="video")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8", action="store_true", help="the layer's FP8 (E4M3) form on the workload's shape")
@@ -305,7 +306,12 @@ def run_ours(args, wl):
     gemm_mean = statistics.mean(gemm_ms)
     gemm_flop = 2 * M * N * K + 2 * M * R * N
     peaks, peaks_kind = load_peaks()
-    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    clock_summary = clocks.summary()
+    # A GEMM that runs under the power cap during the timed loop is a kernel
+    # timed inside a long step: its denominator is the sustained dense rate.
+    sustained = "sw_power_cap" in clock_summary.get("reasons", [])
+    dense_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    sparse_peak = 2.0 * dense_peak
     achieved = gemm_flop / (gemm_mean / 1e3) / 1e12
     traffic = profiled_traffic(wl.name)
     pro_bytes = 2 * M * K + M * K + M * K // 8 + 4 * M + 2 * M * R + 2 * R * K
@@ -328,9 +334,11 @@ def run_ours(args, wl):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": sparse_peak, "unit": "TFLOP/s",
                      "frac": achieved / sparse_peak, "traffic": traffic,
                      "kernel": "rtlynx_gemm_pair_kernel<sparse, 240>",
-                     "peak_note": f"2 x {peaks_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s): "
-                                  "2:4 sparse nominal ratio"},
-        "clocks": clocks.summary(),
+                     "peak_note": f"2 x {peaks_kind} dense bf16 {'sustained' if sustained else 'burst'} "
+                                  f"({dense_peak} TFLOP/s; sustained when the timed loop ran under the power cap): "
+                                  "2:4 sparse nominal ratio",
+                     "frac_of_burst": achieved / (2.0 * peaks["bf16_tflops"])},
+        "clocks": clock_summary,
         # the prologue (both passes) against the HBM roofline: algorithmic bytes
         # are X read, kept values + metadata + s + T written, L_B read once
         "prologue_roofline": {
@@ -350,22 +358,19 @@ def run_ours(args, wl):
 
 
 def profiled_traffic(workload):
-    """DRAM bytes per GEMM launch from the committed ncu summary of this
-    workload, or None when there is none or the kernel source changed since."""
-    path = os.path.join(ROOT, "profiles", f"gemm_sparse_{workload}.md")
+    """DRAM bytes per GEMM launch from the committed ncu counters of this
+    workload (profiles/gemm_sparse_<workload>.json: traffic_bytes_per_launch,
+    kernel_rev), or None when there are none or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", f"gemm_sparse_{workload}.json")
     if not os.path.exists(path):
         return None
-    fields = {}
     with open(path) as f:
-        for line in f:
-            if ":" in line and not line.startswith(("|", "#", " ")):
-                k, v = line.split(":", 1)
-                fields[k.strip()] = v.strip()
+        fields = json.load(f)
     if fields.get("kernel_rev") != kernel_rev():
         return None
     try:
         return int(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, TypeError, ValueError):
         return None
 
 
