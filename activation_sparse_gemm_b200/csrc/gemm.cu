@@ -435,8 +435,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int local = 0; pair_work(local, pair, num_pairs, args, w); ++local) {
             const int buf = local & 1;
             const uint32_t use = static_cast<uint32_t>(local >> 1);
-            if (!warp_wait(&acc_full[buf], use & 1u, err)) break;
-            tc_fence_after();
             int mp, nt;
             tile_coords(w.tile, args, mp, nt);
             const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM + quad * 32;
@@ -444,7 +442,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const uint32_t acc = tmem_base + static_cast<uint32_t>(buf * BN) + lane_addr;
             const bool split = w.unit >= 0;
             float* qw_w = qw_sh + (warp - 2) * BN;  // FP8: this warp's copy of the tile's q_w
+            float qxr = 0.0f;                        // FP8: q_x of this lane's token, loaded once per tile
             if constexpr (FP8) {
+                qxr = args.qx[row0 + lane];
                 // one coalesced pass per tile; zero scales (all-zero channels) and
                 // columns past N apply as 1
                 for (int j = lane; j < BN; j += 32) {
@@ -453,6 +453,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 }
                 __syncwarp();
             }
+            // the scales above do not depend on the accumulator: their loads
+            // overlap the main loop of this tile
+            if (!warp_wait(&acc_full[buf], use & 1u, err)) break;
+            tc_fence_after();
             bool write_y = true;
             const int S = args.tail_split;
             const int tt = w.tile - args.full_tiles;  // index among the split tiles
@@ -573,7 +577,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         }
                     }
                     if constexpr (FP8) {  // dequantise: q_x of the token times q_w of the column
-                        const float qxr = args.qx[row0 + lane];
                         const float4* w4 = reinterpret_cast<const float4*>(qw_w + c);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
