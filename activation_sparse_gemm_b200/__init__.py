@@ -63,7 +63,8 @@ class WsLayout(ctypes.Structure):
 class Schedule(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "prologue_ctas", "prologue_tiles", "prologue_max_segs", "row_blocks", "k_tiles_per_block",
-        "gemm_pairs", "gemm_tiles", "tail_full", "tail_split", "tail_units", "k_stages", "lora_stages")]
+        "gemm_pairs", "gemm_tiles", "tail_full", "tail_split", "tail_units", "k_stages", "lora_stages",
+        "small_path")]
 
 
 def lib() -> ctypes.CDLL:

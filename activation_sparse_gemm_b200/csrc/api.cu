@@ -378,6 +378,13 @@ static int run_layer(DeviceInfo* di, const void* X, const void* W, const void* L
         return RTLYNX_ERR_INVALID_ARG;
     const Workspace ws = carve(workspace, l);
     if (!record(ev_start)) return RTLYNX_ERR_CUDA;
+    if (act == 0 && small_path_fits(d, di->num_sms)) {
+        // one kernel: each CTA pair sparsifies its tokens in shared memory
+        if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
+        if (launch_small(d, X, W, lora ? L_A : nullptr, lora ? L_B : nullptr, ws, Y, di->err_word, stream))
+            return RTLYNX_ERR_CUDA;
+        return record(ev_end) ? RTLYNX_OK : RTLYNX_ERR_CUDA;
+    }
     int rc = run_prologue(d, X, lora ? L_B : nullptr, ws, di->err_word, di->num_sms, stream);
     if (rc) return rc;
     if (!record(ev_mid)) return RTLYNX_ERR_CUDA;
@@ -699,13 +706,17 @@ int rtlynx_schedule_info(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int 
     out->tail_units = d.tail_units;
     out->k_stages = sparse_k_stages(d);
     out->lora_stages = sparse_lora_stages(d);
+    out->small_path = small_path_fits(d, num_sms) ? 1 : 0;
     return RTLYNX_OK;
 }
 
 int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode) {
     if (mode == RTLYNX_MODE_DENSE_SKIP) return (M > 0 && D_in > 0 && D_out > 0) ? 1 : 0;
     if (mode != RTLYNX_MODE_SPARSE || M <= 0 || D_in <= 0 || D_out <= 0 || R < 0 || D_in % 8 || D_out % 8) return 0;
-    return 3;  // streaming sparsify pass, per-token scale pass, GEMM
+    DeviceInfo* di = nullptr;
+    const int sms = current_device(&di) == RTLYNX_OK ? di->num_sms : 148;
+    // one kernel for small problems; else the streaming sparsify pass, the scale pass and the GEMM
+    return small_path_fits(make_dims(M, D_in, D_out, R, sms), sms) ? 1 : 3;
 }
 
 int rtlynx_wait_selftest(int64_t limit_ns, void* stream_) {

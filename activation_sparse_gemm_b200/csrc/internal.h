@@ -158,6 +158,12 @@ Workspace carve(void* base, const WsLayout& l);
 int run_prologue(const Dims& d, const void* X, const void* L_B, const Workspace& ws, int* err, int num_sms,
                  cudaStream_t stream);
 
+// Small problems in one kernel (small.cu): one wave of 256 x 240 tiles,
+// D_in <= 256, R = 0 or R <= 64, bf16, no epilogue activation.
+bool small_path_fits(const Dims& d, int num_sms);
+int launch_small(const Dims& d, const void* X, const void* W, const void* L_A, const void* L_B,
+                 const Workspace& ws, void* Y, int* err, cudaStream_t stream);
+
 int launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t stream);
 int launch_unpack_debug(const Dims& d, const Workspace& ws, void* vals, void* meta, void* s, void* T,
                         cudaStream_t stream);

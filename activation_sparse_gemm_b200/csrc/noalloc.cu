@@ -83,6 +83,9 @@ extern "C" int rtlynx_linear_noalloc(const void* X, const void* W, const void* L
     const WsLayout l = make_ws_layout(d);
     if (l.total > kNoAllocBytes) return RTLYNX_ERR_UNSUPPORTED;  // workspace larger than the static array
     const Workspace ws = carve(scratch, l);
+    if (small_path_fits(d, num_sms))
+        return launch_small(d, X, W, lora ? L_A : nullptr, lora ? L_B : nullptr, ws, Y, err, stream) ? RTLYNX_ERR_CUDA
+                                                                                                  : RTLYNX_OK;
     rc = run_prologue(d, X, lora ? L_B : nullptr, ws, err, num_sms, stream);
     if (rc) return rc;
     if (launch_gemm(d, true, nullptr, W, lora ? L_A : nullptr, ws, Y, 0, num_sms, err, stream))

@@ -102,6 +102,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     return mbar_wait_limit(bar, parity, err, kWaitLimitNs);
 }
 
+// The same wait with acquire semantics at cluster scope: for barriers the
+// other CTA of the pair arrives on (with release at cluster scope) after
+// writing its shared memory.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspended tries, like mbar_wait_limit: the thread wakes when the phase
+// completes, and reads the error word (a global load) only between tries.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* err) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(bar, parity, kSuspendHintNs)) {
+        if (error_seen(err)) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(err, RTLYNX_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- TMA / bulk copies
 // Programmatic dependent launch: the kernel that follows in the stream may
 // start once every CTA of this grid has called launch_dependents (or exited);
@@ -276,6 +305,23 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                      reinterpret_cast<uint64_t>(map)),
                  "r"(smem_u32(src)), "r"(x), "r"(y)
                  : "memory");
+}
+
+// Contiguous shared -> global copy (16-byte aligned addresses, size multiple of 16), bulk-group completion.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+// Named barrier over `threads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Arrives on a named barrier without waiting for it (the waiting side calls named_barrier).
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t threads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }

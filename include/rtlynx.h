@@ -244,16 +244,23 @@ int rtlynx_linear_noalloc(const void* X, const void* W, const void* L_A, const v
  *                      later tile is cut along its stages into tail_split
  *                      parts (tail_units parts in all, one per pair)
  *   k_stages, lora_stages  pipeline stages of one tile (main loop, LoRA-up)
+ *   small_path         1 when the problem is one wave of 256 x 240 tiles with
+ *                      D_in <= 256 and R = 0 or R <= 64: the call is then one
+ *                      kernel whose CTA pairs sparsify their own tokens in
+ *                      shared memory (the fields above describe the general
+ *                      form it replaces)
  * RTLYNX_ERR_INVALID_ARG for invalid sizes or a NULL out. */
 typedef struct {
     int64_t prologue_ctas, prologue_tiles, prologue_max_segs, row_blocks, k_tiles_per_block;
     int64_t gemm_pairs, gemm_tiles, tail_full, tail_split, tail_units, k_stages, lora_stages;
+    int64_t small_path;  /* 1: the call runs as one kernel (small problems, see above) */
 } rtlynx_schedule;
 int rtlynx_schedule_info(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int num_sms, rtlynx_schedule* out);
 
-/* Number of kernels one rtlynx_linear call with these sizes launches (0 for
- * invalid sizes): the sparse path launches its prologue kernel(s) and the GEMM,
- * the dense-skip path the GEMM alone. */
+/* Number of kernels one rtlynx_linear call with these sizes launches on the
+ * current device (0 for invalid sizes): the sparse path launches its two
+ * sparsify kernels and the GEMM, or one kernel where the problem takes the
+ * small path (rtlynx_schedule.small_path); the dense-skip path the GEMM alone. */
 int rtlynx_kernel_launches(int64_t M, int64_t D_in, int64_t D_out, int64_t R, int mode);
 
 /* Self-test of the device-side failure detection: launches one thread that

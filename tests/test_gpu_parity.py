@@ -169,9 +169,29 @@ def test_sparsify_small(M, K, R):
     assert frac_same > 0.99
 
 
+def unpack_workspace(ws, lay, M, K, R):
+    """The kept values, metadata, s and T straight from a workspace, the
+    metadata unpacked with the documented tensor-memory mapping (independently
+    of the library's unpack kernel)."""
+    raw = ws.cpu().numpy()
+    chunks = raw[lay.meta:lay.meta + (lay.M_pad // 128) * lay.k_chunks * 2048].reshape(
+        lay.M_pad // 128, lay.k_chunks, 2048)
+    words = chunks.view(np.uint32).reshape(lay.M_pad // 128, lay.k_chunks, 128, 4)  # [mb, kc, lane, col]
+    m = np.arange(M)
+    mb, mm = m // 128, m % 128
+    m0, m1, m2 = mm % 8, (mm // 8) % 2, mm // 16
+    k = 4 * np.arange(K // 4)
+    kc, kk = k // 128, k % 128
+    k0, k1, k2 = kk % 16, (kk // 16) % 2, kk // 32
+    w = words[mb[:, None], kc[None, :], (m0[:, None] + 8 * k1[None, :] + 16 * m2[:, None]), k2[None, :]]
+    meta = ((w >> (16 * m1[:, None] + 4 * (k0[None, :] // 4))) & 0xF).astype(np.uint8)
+    vals = raw[lay.vals:lay.vals + lay.M_pad * lay.Kc_pad * 2].view(np.uint16).reshape(lay.M_pad, lay.Kc_pad)
+    s = raw[lay.s:lay.s + lay.M_pad * 4].view(np.float32)
+    T = raw[lay.T:lay.T + lay.M_pad * lay.R_pad * 2].view(np.uint16).reshape(lay.M_pad, lay.R_pad) if R else None
+    return meta, vals, s, T
+
+
 def test_sparsify_raw_workspace_layout():
-    """Unpack the metadata straight from the workspace with the documented
-    tensor-memory mapping (independently of the library's unpack kernel)."""
     import torch
     M, K, N, R = 200, 384, 64, 32
     X, W, L_A, L_B = make_custom(M, K, N, R, seed=5)
@@ -180,25 +200,49 @@ def test_sparsify_raw_workspace_layout():
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     rl.rtlynx_linear_ws(dev(X), dev(W), dev(L_A), dev(L_B), Y, M, K, N, R, rl.MODE_SPARSE, ws, lay.total)
     assert rl.rtlynx_stream_status() == rl.OK
-    raw = ws.cpu().numpy()
-    chunks = raw[lay.meta:lay.meta + (lay.M_pad // 128) * lay.k_chunks * 2048].reshape(
-        lay.M_pad // 128, lay.k_chunks, 2048)
-    words = chunks.view(np.uint32).reshape(lay.M_pad // 128, lay.k_chunks, 128, 4)  # [mb, kc, lane, col]
+    meta, vals, _, _ = unpack_workspace(ws, lay, M, K, R)
     rmeta, rvals, rs = oracle.sparsify(X)
-    meta = np.empty_like(rmeta)
-    for m in range(M):
-        mb, mm = divmod(m, 128)
-        m0, m1, m2 = mm % 8, (mm // 8) % 2, mm // 16
-        for g in range(K // 4):
-            k = 4 * g
-            kc, kk = divmod(k, 128)
-            k0, k1, k2 = kk % 16, (kk // 16) % 2, kk // 32
-            w = int(words[mb, kc, m0 + 8 * k1 + 16 * m2, k2])
-            meta[m, g] = (w >> (16 * m1 + 4 * (k0 // 4))) & 0xF
     assert (meta == rmeta).all()
-    vals = raw[lay.vals:lay.vals + lay.M_pad * lay.Kc_pad * 2].view(np.uint16).reshape(lay.M_pad, lay.Kc_pad)
     assert (bf16_ulp_dist(vals[:M, :K // 2], rvals) <= 1).all()
     assert (vals[M:] == 0).all() and (vals[:, K // 2:] == 0).all()
+
+
+@pytest.mark.parametrize("M,K,N,R", [(128, 256, 256, 64), (200, 256, 64, 32), (127, 72, 264, 16), (1, 64, 8, 8),
+                                     (5000, 136, 264, 16), (300, 192, 40, 0), (256, 256, 17 * 240, 64)])
+def test_small_path_one_kernel(M, K, N, R):
+    """Problems of one wave of tiles with D_in <= 256 run as one kernel whose
+    CTA pairs sparsify their tokens in shared memory.  Y meets the bar, and
+    the kept values, metadata, s and T it leaves in the workspace meet the
+    prologue's bars (metadata bit-exact, values within 1 ulp and exact where
+    s is, s within 2 ulp)."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert rl.rtlynx_schedule_info(M, K, N, R, sms).small_path == 1
+    assert rl.rtlynx_kernel_launches(M, K, N, R, rl.MODE_SPARSE) == 1
+    X, W, L_A, L_B = make_custom(M, K, N, R if R else 8, seed=400 + M + K)
+    if R == 0:
+        L_A = L_B = None
+    lay = rl.rtlynx_workspace_layout(M, K, N, R)
+    ws = torch.full((lay.total,), 0xFF, dtype=torch.uint8, device="cuda")  # stale bytes must not matter
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    rl.rtlynx_linear_ws(dev(X), dev(W), None if R == 0 else dev(L_A), None if R == 0 else dev(L_B), Y, M, K, N, R,
+                        rl.MODE_SPARSE, ws, lay.total)
+    assert rl.rtlynx_stream_status() == rl.OK
+    assert_y_close(host_bits(Y), oracle.linear(X, W, L_A, L_B), f"small path {M}x{K}x{N} R={R}")
+    meta, vals, s, T = unpack_workspace(ws, lay, M, K, R)
+    rmeta, rvals, rs = oracle.sparsify(X)
+    assert (meta == rmeta).all(), "metadata differs"
+    assert (ulp_dist_f32(s[:M], rs) <= 2).all(), "s differs by more than 2 ulp"
+    assert (bf16_ulp_dist(vals[:M, :K // 2], rvals) <= 1).all(), "values differ by more than 1 bf16 ulp"
+    same = s[:M] == rs
+    assert (vals[:M, :K // 2][same] == rvals[same]).all()
+    assert (vals[M:] == 0).all() and (vals[:, K // 2:] == 0).all()
+    if R:
+        _, Tref = oracle.linear(X, np.zeros((8, K), np.uint16), np.zeros((8, R), np.uint16), L_B, want_T=True)
+        err = np.abs(f64(T[:M, :R]) - Tref)
+        scale = np.abs(bf16_bits_to_f32(X)) @ np.abs(bf16_bits_to_f32(L_B)).T
+        assert (err <= 2.0 ** -8 * np.abs(Tref) + 2e-5 * scale.astype(np.float64) + 1e-30).all(), "T out of tolerance"
+        assert (T[:M, R:] == 0).all()
 
 
 # ------------------------------------------------------------------ the fused layer
