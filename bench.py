@@ -346,19 +346,19 @@ def run_ours(args, wl):
                                   "2:4 sparse nominal ratio",
                      "frac_of_burst": achieved / (2.0 * peaks["bf16_tflops"])},
         "clocks": clock_summary,
+    }
+    if not small:
         # the prologue (both passes) against the HBM roofline: algorithmic bytes
         # are X read, kept values + metadata + s + T written, L_B read once
-        "prologue_roofline": {
-            "bound": "hbm", "bytes": pro_bytes, "achieved": pro_bytes / (statistics.mean(pro_ms) / 1e3) / 1e9,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": pro_bytes / (statistics.mean(pro_ms) / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "note": "phase time from the split loop (an event between prologue and GEMM)"},
-    }
-    if small:
+        pro_gbs = pro_bytes / (statistics.mean(pro_ms) / 1e3) / 1e9
+        line["prologue_roofline"] = {
+            "bound": "hbm", "bytes": pro_bytes, "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": pro_gbs / peaks["hbm_gbs"],
+            "note": "phase time from the split loop (an event between prologue and GEMM)"}
+    else:
         # one kernel: sparsify, both GEMMs and the epilogue; its bytes (X, W,
         # L_A, L_B read; Y and the workspace copy written) over the call time
         # show how far a problem this small is from any bandwidth roofline
-        del line["prologue_roofline"]
         one_bytes = 2 * M * K + 2 * N * K + 2 * (N * R + R * K) + 2 * M * N + pro_bytes - 2 * M * K - 2 * R * K
         line["small_path"] = {"kernel": "rtlynx_small_kernel", "launches_per_call": 1, "bytes": one_bytes,
                               "achieved_gbs": one_bytes / (ms / 1e3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
