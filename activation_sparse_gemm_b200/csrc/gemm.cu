@@ -444,12 +444,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             float* qw_w = qw_sh + (warp - 2) * BN;  // FP8: this warp's copy of the tile's q_w
             float qxr = 0.0f;                        // FP8: q_x of this lane's token, loaded once per tile
             if constexpr (FP8) {
-                qxr = args.qx[row0 + lane];
-                // one coalesced pass per tile; zero scales (all-zero channels) and
-                // columns past N apply as 1
-                for (int j = lane; j < BN; j += 32) {
-                    const float v = col0 + j < args.N ? args.qw[col0 + j] : 1.0f;
-                    qw_w[j] = v > 0.0f ? v : 1.0f;
+                qxr = __ldg(args.qx + row0 + lane);
+                // one coalesced pass per tile, every load in flight before the
+                // first store (the stores go through a generic pointer, so loads
+                // interleaved with them would each wait out their own latency);
+                // zero scales (all-zero channels) and columns past N apply as 1
+                constexpr int kQw = (BN + 31) / 32;
+                float qv[kQw];
+#pragma unroll
+                for (int i = 0; i < kQw; ++i) {
+                    const int j = lane + 32 * i;
+                    qv[i] = (j < BN && col0 + j < args.N) ? __ldg(args.qw + col0 + j) : 1.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < kQw; ++i) {
+                    const int j = lane + 32 * i;
+                    if (j < BN) qw_w[j] = qv[i] > 0.0f ? qv[i] : 1.0f;
                 }
                 __syncwarp();
             }
