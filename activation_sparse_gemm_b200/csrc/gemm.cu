@@ -16,8 +16,9 @@
 //               stages carry the compressed S(X) tile, the W tile and the 2 KB
 //               metadata chunk of their 128 K; then come the LoRA stages (T
 //               tile and L_A tile).
-//   warp 1      tensor-memory owner; in the leader CTA one thread issues every
-//               MMA of the pair: tcgen05.mma.sp (K = 32 logical per instruction)
+//   warp 1      tensor-memory owner; in the leader CTA the warp runs the issue
+//               loop and one elected lane issues every MMA of the pair:
+//               tcgen05.mma.sp (K = 32 logical per instruction)
 //               with the metadata moved into tensor memory by tcgen05.cp, and
 //               dense tcgen05.mma for the LoRA stages into the SAME accumulator,
 //               so T L_A^T never leaves the chip.  Its commits arrive on the
@@ -348,7 +349,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (leader && lane == 0) {
+        if (leader) {
+            // The whole warp runs the issue loop, so its descriptors and counters
+            // are warp-uniform values; one elected lane (always the same one, so
+            // its commits track all of its MMAs) issues the tcgen05 instructions.
+            // Measured against lane 0 running the loop alone: 2-4% faster GEMMs
+            // (qkv sparse 105.4 -> 102.0 us, dense-skip 146.9 -> 141.3 us).
             const uint32_t idesc_main = FP8 ? make_idesc_e4m3(2 * kBM, BN, true) : make_idesc_bf16(2 * kBM, BN, SPARSE);
             const uint32_t idesc_dense = make_idesc_bf16(2 * kBM, BN, false);
             // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the
@@ -369,14 +375,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int local = 0; ok && pair_work(local, pair, num_pairs, args, w); ++local) {
                 const int buf = local & 1;
                 const uint32_t use = static_cast<uint32_t>(local >> 1);
-                if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, err)) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, err))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
                 for (int kt = w.kb; kt < w.ke; ++kt) {
-                    if (!mbar_wait(&full[stage], phase, err)) {
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[stage], phase, err))) {
                         ok = false;
                         break;
                     }
@@ -384,7 +390,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const uint64_t a = descA0 + off;
                     const uint64_t b = descB0 + off;
                     const uint32_t acc = kt != w.kb;  // the item's first stage starts the accumulator
-                    if (kt < args.k_stages) {
+                    if (!elect_one()) {
+                        // the other lanes only keep the loop's state
+                    } else if (kt < args.k_stages) {
                         if constexpr (FP8) {
                             // two metadata chunks -> columns [meta, meta + 8); MMA j reads columns meta + 2j, + 2j + 1
                             tmem_cp_128x128b_pair(tmem_meta, descE0 + off);
@@ -411,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         mma_f16_pair(d, a + 4, b + 4, idesc_dense, 1u);
                         mma_f16_pair(d, a + 6, b + 6, idesc_dense, 1u);
                     }
-                    tc_commit_pair_mc(&empty[stage], 0x3);
+                    if (elect_one()) tc_commit_pair_mc(&empty[stage], 0x3);
                     off += kStageStep;
                     if (++stage == G::STAGES) {
                         stage = 0;
@@ -420,12 +428,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair_mc(&acc_full[buf], 0x3);
+                if (elect_one()) tc_commit_pair_mc(&acc_full[buf], 0x3);
             }
             // Every MMA of the pair has finished before tensor memory is freed.
-            tc_commit_pair_mc(done_bar, 0x1);
+            if (elect_one()) tc_commit_pair_mc(done_bar, 0x1);
             mbar_wait(done_bar, 0, nullptr);
         }
+        __syncwarp();
     } else {
         const int quad = warp & 3;  // warps 2..5 own tensor-memory lane quadrants 2,3,0,1
         const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
