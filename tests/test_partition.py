@@ -100,3 +100,36 @@ def test_schedule_rejects_bad_arguments():
         rl.rtlynx_schedule_info(16, 60, 64, 0, 148)
     with pytest.raises(rl.RtlynxError):
         rl.rtlynx_schedule_info(16, 64, 64, 0, 1)
+
+
+def test_small_path_selection():
+    """The one-kernel small path: the output is one wave of 256 x 240 tiles
+    (at most one CTA pair per two SMs), D_in <= 256 and R <= 64; anything
+    else takes the general three-kernel path."""
+    def small(M, K, N, R, sms=148):
+        return rl.rtlynx_schedule_info(M, K, N, R, sms).small_path
+
+    assert small(128, 256, 256, 64) == 1          # the tiny workload
+    assert small(4096, 3072, 9216, 64) == 0       # qkv
+    assert small(128, 264, 256, 64) == 0          # D_in past 256
+    assert small(128, 256, 256, 72) == 0          # R past 64
+    assert small(128, 256, 256, 0) == 1           # no LoRA
+    assert small(1, 8, 8, 8) == 1
+    # one wave: 74 pairs on 148 SMs (row pairs of 256 tokens x column tiles of 240)
+    assert small(256 * 74, 256, 240, 16) == 1
+    assert small(256 * 74 + 1, 256, 240, 16) == 0
+    assert small(256 * 37, 256, 480, 16) == 1
+    assert small(256 * 37, 256, 488, 16) == 0
+    assert small(256 * 37, 256, 480, 16, sms=72) == 0
+    # the ABI's launch count follows the same rule (148 SMs where no GPU is present)
+    if rl.rtlynx_schedule_info(128, 256, 256, 64, 148).small_path == 1 and not _has_gpu():
+        assert rl.rtlynx_kernel_launches(128, 256, 256, 64, rl.MODE_SPARSE) == 1
+        assert rl.rtlynx_kernel_launches(4096, 3072, 9216, 64, rl.MODE_SPARSE) == 3
+
+
+def _has_gpu():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
