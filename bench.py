@@ -264,9 +264,12 @@ def run_ours(args, wl):
         pro_ms = [a.elapsed_time(b) for a, b, c in pevs]
         gemm_ms = [b.elapsed_time(c) for a, b, c in pevs]
 
-    # same-run comparisons (not part of the headline value)
+    # same-run comparisons (not part of the headline value), each with its own
+    # clock record: long dense loops can run into the power cap
     for _ in range(3):
         torch.matmul(Xd, Wd.t(), out=Y)
+    cublas_clocks = ClockSampler(device)
+    cublas_clocks.start()
     cublas_pairs = []
     for _ in range(args.steps):
         flush.fill_(1)
@@ -275,10 +278,13 @@ def run_ours(args, wl):
         b = ev()
         cublas_pairs.append((a, b))
     torch.cuda.synchronize()
+    cublas_clocks.stop()
     cublas_ms = statistics.mean(a.elapsed_time(b) for a, b in cublas_pairs)
     ours_dense_pairs = []
     for _ in range(max(3, args.warmup)):
         sparse_step(mode=rl.MODE_DENSE_SKIP)
+    dense_clocks = ClockSampler(device)
+    dense_clocks.start()
     for _ in range(args.steps):
         flush.fill_(1)
         a = ev()
@@ -286,6 +292,7 @@ def run_ours(args, wl):
         b = ev()
         ours_dense_pairs.append((a, b))
     torch.cuda.synchronize()
+    dense_clocks.stop()
     ours_dense_ms = statistics.mean(a.elapsed_time(b) for a, b in ours_dense_pairs)
 
     # end to end through the host-buffer entry point
@@ -346,6 +353,8 @@ def run_ours(args, wl):
                                   "2:4 sparse nominal ratio",
                      "frac_of_burst": achieved / (2.0 * peaks["bf16_tflops"])},
         "clocks": clock_summary,
+        "comparison_clocks": {"cublas_dense": _clock_brief(cublas_clocks.summary()),
+                              "ours_dense_skip": _clock_brief(dense_clocks.summary())},
     }
     if not small:
         # the prologue (both passes) against the HBM roofline: algorithmic bytes
@@ -371,6 +380,11 @@ def run_ours(args, wl):
         print(json.dumps(line), flush=True)
     rdist.shutdown()
     return 0
+
+
+def _clock_brief(summary):
+    """Median SM MHz and the throttle reasons seen, from a ClockSampler summary."""
+    return {"sm_mhz": summary.get("sm_mhz"), "reasons": summary.get("reasons", [])}
 
 
 def profiled_traffic(workload):
