@@ -270,16 +270,23 @@ def run_ours(args, wl):
         torch.matmul(Xd, Wd.t(), out=Y)
     cublas_clocks = ClockSampler(device)
     cublas_clocks.start()
-    cublas_pairs = []
+    # cuBLAS and our sparse call alternate, each after an L2 flush, so that both
+    # run in the same power and clock state: the speedup comes from this loop
+    cublas_pairs, ours_pairs = [], []
     for _ in range(args.steps):
         flush.fill_(1)
         a = ev()
         torch.matmul(Xd, Wd.t(), out=Y)
         b = ev()
         cublas_pairs.append((a, b))
+        flush.fill_(1)
+        es = [ev(), ev()]
+        sparse_step(es[0], None, es[1])
+        ours_pairs.append(es)
     torch.cuda.synchronize()
     cublas_clocks.stop()
     cublas_ms = statistics.mean(a.elapsed_time(b) for a, b in cublas_pairs)
+    ours_alt_ms = statistics.mean(a.elapsed_time(b) for a, b in ours_pairs)
     ours_dense_pairs = []
     for _ in range(max(3, args.warmup)):
         sparse_step(mode=rl.MODE_DENSE_SKIP)
@@ -332,7 +339,8 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3,
-        "speedup_vs_dense_bf16": cublas_ms / ms, "dense_bf16_cublas_us": cublas_ms * 1e3,
+        "speedup_vs_dense_bf16": cublas_ms / ours_alt_ms, "dense_bf16_cublas_us": cublas_ms * 1e3,
+        "us_per_call_alternating": ours_alt_ms * 1e3,
         "ours_dense_skip_us": ours_dense_ms * 1e3,
         "phases_us": ({"one_kernel": gemm_mean * 1e3} if small else
                       {"sparsify_prologue": statistics.mean(pro_ms) * 1e3, "sparse_gemm_lora": gemm_mean * 1e3}),
@@ -353,7 +361,7 @@ def run_ours(args, wl):
                                   "2:4 sparse nominal ratio",
                      "frac_of_burst": achieved / (2.0 * peaks["bf16_tflops"])},
         "clocks": clock_summary,
-        "comparison_clocks": {"cublas_dense": _clock_brief(cublas_clocks.summary()),
+        "comparison_clocks": {"cublas_and_ours_alternating": _clock_brief(cublas_clocks.summary()),
                               "ours_dense_skip": _clock_brief(dense_clocks.summary())},
     }
     if not small:
